@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark: ADA paged decode KV tokens/s on B200 (one JSON line on rank 0).
+
+One step = the whole decode hot path for one batch: append the step's new
+token (key and value) of every sequence through spkv_encode_keys, then
+spkv_decode_attention over all ctx tokens of every sequence (split kernel +
+merge kernel).  Default workload: Llama-3-8B-shaped layer decode, B = 8,
+32 query / 8 kv heads, d = 128, ctx = 32768, page 16, b = 4 (673 MB of codes,
+radii and values per step: far larger than the 126 MB L2, so no flush is
+needed between steps).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl spkv|reference]
+
+N > 1 is launched by torchrun, one rank per GPU; every rank decodes its own
+batch (independent sequences: weak scaling, no collective on the data path);
+the step time is the max over ranks.  --impl reference times the fp64 CPU
+oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _dist():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ GPU arm
+def run_spkv(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    import compressed_kv_decode_ada_b200 as spkv
+    from compressed_kv_decode_ada_b200 import synthetic, workload
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    cfg = dict(synthetic.CONFIGS[args.config])
+    cfg["seed"] = int(cfg["seed"]) + 1000 * rank  # each rank: its own independent batch
+    wl = synthetic.make_workload(cfg, device=dev)
+    cache = workload.build_cache(wl)
+    B, Hq, Hkv = wl.B, wl.Hq, wl.Hkv
+    ctx = wl.ctx_tensor(dev)
+    max_ctx = wl.max_ctx
+    splits = spkv.default_splits(B, Hkv, max_ctx) if args.splits == 0 else args.splits
+    ws = spkv.alloc_workspace(B, Hq, Hkv, max_ctx, splits, device=dev)
+    out = torch.empty((B, Hq, 128), dtype=torch.float32, device=dev)
+    # the step's new token: the last context position of every sequence
+    last = torch.as_tensor((wl.ctx - 1).astype(np.int32), device=dev)
+    new_idx = torch.as_tensor(wl.seq_off[1:] - 1, device=dev).long()
+    new_k = wl.keys[new_idx].unsqueeze(1).contiguous()     # [B, 1, Hkv, 128]
+    new_v = wl.values[new_idx].unsqueeze(1).contiguous()
+    stream = torch.cuda.current_stream(dev)
+
+    def step(q, k, v, o):
+        spkv.encode_keys(cache, k, last, wl.block_table, values=v, stream=stream)
+        spkv.decode_attention(cache, q, wl.block_table, ctx, max_ctx, out=o, ws=ws, num_splits=splits,
+                              stream=stream)
+
+    for _ in range(args.warmup):
+        step(wl.q, new_k, new_v, out)
+    torch.cuda.synchronize(dev)
+    if cache.error_flags():
+        raise RuntimeError(f"device error flags {cache.error_flags():#x}")
+
+    # ---------------- timed region: K steps, per-step events around the decode call
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            spkv.encode_keys(cache, new_k, last, wl.block_table, values=new_v, stream=stream)
+            ev_dec[i][0].record(stream)
+            spkv.decode_attention(cache, wl.q, wl.block_table, ctx, max_ctx, out=out, ws=ws, num_splits=splits,
+                                  stream=stream)
+            ev_dec[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    total_ms = t_start.elapsed_time(t_end)
+    dec_ms = sum(a.elapsed_time(b) for a, b in ev_dec) / args.steps
+    ms_step = total_ms / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step, dec_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, dec_ms = float(t[0]), float(t[1])
+    clocks = clk.summary()
+
+    # ---------------- end to end through the public API with host buffers
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    q_h = wl.q.cpu().pin_memory()
+    k_h, v_h = new_k.cpu().pin_memory(), new_v.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_d, k_d, v_d = torch.empty_like(wl.q), torch.empty_like(new_k), torch.empty_like(new_v)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(e2e_steps + 2):
+        if i == 2:
+            e0.record(stream)
+        q_d.copy_(q_h, non_blocking=True)
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        step(q_d, k_d, v_d, out)
+        out_h.copy_(out, non_blocking=True)
+        stream.synchronize()  # the host reads the step's result
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    if cache.error_flags():
+        raise RuntimeError(f"device error flags {cache.error_flags():#x}")
+
+    extras = {}
+    if rank == 0 and args.compare:
+        extras = compare_paths(args, spkv, workload, wl, cache, ctx, max_ctx, splits, ws, stream, dev)
+
+    tokens = wl.kv_tokens
+    bytes_step = synthetic.ada_step_bytes(wl)
+    result = None
+    if rank == 0:
+        peak, peak_kind = _peaks()
+        achieved = bytes_step / (dec_ms * 1e-3) / 1e9
+        traffic = _committed_traffic(args.config)
+        h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
+        d2h = out_h.numel() * out_h.element_size()
+        result = {
+            "metric": "ADA decode KV tokens/s on 1 B200; achieved HBM GB/s as % of peak",
+            "value": tokens * world / (ms_step * 1e-3),
+            "unit": "KV tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded: N(0,1) bf16 keys x log-normal channel scales with 4 outliers, RoPE base "
+                    "500000; N(0,1) bf16 values and queries)",
+            "config": {"workload": wl.name, "B": B, "num_q_heads": Hq, "num_kv_heads": Hkv, "ctx": int(max_ctx),
+                       "page": 16, "bits": sorted(set(int(b) for b in wl.page_bits)), "splits": splits,
+                       "kv_tokens_per_step": tokens, "algorithmic_bytes_per_step": bytes_step,
+                       "l2": "no flush: the step streams %.0f MB > 126 MB L2" % (bytes_step / 1e6),
+                       "step": "append 1 token/sequence (spkv_encode_keys) + spkv_decode_attention",
+                       "parallelism": f"dp{world} (independent batches)"},
+            "roofline": {"bound": "hbm", "kernel": "spkv_decode_attention (split + merge kernels)",
+                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak, "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS,
+                         "traffic": traffic, "decode_ms": dec_ms},
+            "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks,
+        }
+        if extras:
+            result["comparison"] = extras
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def compare_paths(args, spkv, workload, wl, cache, ctx, max_ctx, splits, ws, stream, dev):
+    """Untimed-in-the-headline comparison: dense bf16 and decompress-then-dot
+    decode of the same batch (same split count), and bulk encode throughput."""
+    import torch
+
+    from compressed_kv_decode_ada_b200 import synthetic
+
+    n = max(5, args.compare_steps)
+    res = {}
+
+    def timeit(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n
+
+    tokens = wl.kv_tokens
+    ada_ms = timeit(lambda: spkv.decode_attention(cache, wl.q, wl.block_table, ctx, max_ctx, ws=ws,
+                                                  num_splits=splits, stream=stream))
+    res["ada_decode_ms"] = ada_ms
+    kp, vp = workload.dense_pages(wl)
+    dense_ms = timeit(lambda: spkv.dense_decode(kp, vp, wl.q, wl.block_table, ctx, max_ctx, ws=ws,
+                                                num_splits=splits, stream=stream))
+    res["dense_decode_ms"] = dense_ms
+    res["dense_tokens_per_s"] = tokens / (dense_ms * 1e-3)
+    res["dense_achieved_gbs"] = synthetic.dense_step_bytes(wl) / (dense_ms * 1e-3) / 1e9
+    del kp
+    ks = torch.empty_like(cache.v_pages)
+    dtd_ms = timeit(lambda: spkv.decompress_then_dot(cache, ks, wl.q, wl.block_table, ctx, max_ctx, ws=ws,
+                                                     num_splits=splits, stream=stream))
+    res["decompress_then_dot_ms"] = dtd_ms
+    res["decompress_then_dot_tokens_per_s"] = tokens / (dtd_ms * 1e-3)
+    res["ada_speedup_vs_dense"] = dense_ms / ada_ms
+    res["ada_speedup_vs_decompress_then_dot"] = dtd_ms / ada_ms
+    del ks, vp
+    # bulk encode (prefill) of every context key and value
+    enc_ms = timeit(lambda: workload.prefill(cache, wl))
+    res["encode_ms"] = enc_ms
+    res["encode_keys_per_s"] = tokens * wl.Hkv / (enc_ms * 1e-3)
+    res["encode_unit"] = "(token, kv head) keys/s, with values"
+    res["resident_bytes_per_token"] = {"ada": cache.resident_bytes() / tokens,
+                                       "dense_bf16": 2 * wl.Hkv * 256.0}
+    return res
+
+
+def _committed_traffic(config):
+    """ncu DRAM bytes per launch of the ADA split kernel, from the committed
+    profile summary, if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    src = os.path.join(ROOT, "compressed_kv_decode_ada_b200", "csrc", "decode.cu")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    ent = d.get(str(config))
+    if not ent or ent.get("decode_cu_sha256_16") != sha:
+        return None
+    return ent.get("dram_bytes_per_step")
+
+
+# ------------------------------------------------------------ CPU oracle arm
+def cpu_oracle(args, budget_s: float):
+    """Time the fp64 oracle's decode (ADA attention from codes) on host cores
+    over (sequence, kv head) groups of the same workload, one group per thread;
+    the keys are encoded by the oracle beforehand (untimed).  Returns the line's
+    cpu_baseline dict."""
+    import torch
+
+    import oracle
+    from compressed_kv_decode_ada_b200 import synthetic
+
+    cfg = dict(synthetic.CONFIGS[args.config])
+    wl = synthetic.make_workload(cfg, device="cpu", B=min(cfg["B"], 2))
+    cores = _cores()
+    groups = [(b, h) for b in range(wl.B) for h in range(wl.Hkv)]
+    # tokens per group sized so the timed part stays within the budget
+    per_tok_s = 6e-6 * wl.G / 4 + 4e-6
+    T = int(min(wl.ctx.min(), max(256, budget_s * cores / max(1, len(groups)) / per_tok_s)))
+    T = max(16, (T // 16) * 16)
+    prepared = []
+    for b, h in groups[:max(1, cores)]:
+        keys = wl.keys_bits(b, h)[:T]
+        bits = wl.token_bits(b)[:T]
+        L, D = float(wl.rad_lo[h]), float(wl.rad_step[h])
+        codes, rc = oracle.encode(keys, bits, L, D)
+        prepared.append((wl.q_bits(b, h), codes, bits, rc, L, D, wl.values_bits(b, h)[:T]))
+    # repeat whole passes over the sample until the budget is spent (at least one)
+    passes = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.map_groups(lambda a: oracle.ada_group(*a), prepared, threads=cores)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s:
+            break
+    token_heads = T * len(prepared) * passes
+    value = token_heads / wl.Hkv / dt
+    del torch
+    return {"value": value, "unit": "KV tokens/s", "cores": min(cores, len(prepared)), "kind": "oracle",
+            "sample": f"{passes} passes over {len(prepared)} (sequence, kv head) groups x {T} tokens of "
+                      f"{wl.name} (G={wl.G}, b=4); KV tokens = token-heads / {wl.Hkv}; {dt:.1f} s"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="spkv", choices=["spkv", "reference"])
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--compare", type=int, default=1)
+    ap.add_argument("--compare-steps", type=int, default=50)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = _dist()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cb = cpu_oracle(args, args.cpu_budget)
+        from compressed_kv_decode_ada_b200 import synthetic
+
+        wl_cfg = synthetic.CONFIGS[args.config]
+        line = {"metric": "ADA decode KV tokens/s on 1 B200; achieved HBM GB/s as % of peak", "impl": "reference",
+                "value": cb["value"], "unit": "KV tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": wl_cfg["name"]}, "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "KV tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    res = run_spkv(args, rank, world, local)
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            res["cpu_baseline"] = cpu_oracle(args, args.cpu_budget)
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

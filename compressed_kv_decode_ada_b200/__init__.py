@@ -1,0 +1,11 @@
+"""compressed_kv_decode_ada_b200: Spherical KV angle-domain attention (ADA)
+paged decode on NVIDIA B200 (sm_100a).
+
+The compute lives in libspkv.so (C ABI, include/spkv.h); this package is its
+thin Python binding plus seeded synthetic workloads.  Importing it fails
+loudly when the CUDA library has not been built.
+"""
+from ._lib import LIB_PATH, SpkvError, lib  # noqa: F401
+from .cache import SpkvCache  # noqa: F401
+from .ops import (alloc_workspace, debug_logits, decode_attention, decompress_then_dot,  # noqa: F401
+                  default_splits, dense_decode, encode_keys, workspace_bytes)

@@ -1,0 +1,286 @@
+// encode.cu -- spkv_encode_keys: bf16 keys -> (uint8 log radius code, b-bit
+// angle codes) appended to their page slots through the block table.
+//
+// Method: "SPHERICAL KV: Angle-Domain Attention and Rate-Distortion Retention
+// for Efficient Long-Context Inference", technical summary section 2.1
+// ("spherical parametrisation": r = ||k||, phi = Phi(k^); ADA "stores
+// quantised radii and packed angle codes") and 2.3 ("maps dense keys to
+// spherical codes ... stores them in a compressed format").
+//
+// Every code is decided in fp64 without evaluating any angle: the squares of
+// bf16 inputs are exact in fp64, and
+//   phi_i >= theta_k  <=>  x_i <= sqrt(S_i) cos(theta_k)
+// (S_i = sum_{j >= i} x_j^2) is decided from x_i^2 versus S_i cos^2(theta_k)
+// plus the signs.  The code is the largest k whose edge theta_k the angle
+// reaches (binary search over the 2^b - 1 edges), i.e. floor(phi 2^b / pi)
+// clamped to 2^b - 1 -- ties go to the upper cell.  The azimuth (angle 127,
+// range [0, 2 pi)) uses the same test on (x_126, x_127) with the half-plane
+// given by the sign of x_127.  The radius code uses fp64 log2.
+#include "spkv_common.cuh"
+
+namespace spkv {
+namespace {
+
+constexpr int kEncThreads = 256;
+constexpr int kEncWarps = kEncThreads / 32;
+
+struct EncodeParams {
+  uint8_t *arena;
+  uint64_t arena_bytes;
+  const spkv_page_hdr *hdr;
+  const float *rad_lo, *rad_step;
+  uint16_t *v_pages;
+  uint32_t *err;
+  int Hkv, num_pages;
+  const uint16_t *keys, *values;
+  const int32_t *start_pos, *block_table;
+  int B, n_new, max_pages;
+  int64_t items;  // B * n_new * Hkv
+};
+
+// Shared tables: squared cosines of the cell edges, per tier.
+//   polar   edge k of b bits: theta = k pi / 2^b          (k in [0, 2^b))
+//   azimuth edge k of b bits: theta = k 2 pi / 2^b        (k in [0, 2^b))
+struct EncodeSmem {
+  double pol_c2[kLutEntries];
+  double az_c2[kLutEntries];
+  uint8_t codes[kEncWarps][128];
+};
+
+// phi >= theta_k for a polar angle, given x = x_i, S = S_i (S > 0), the edge's
+// squared cosine c2 and whether its cosine is non-negative.
+__device__ __forceinline__ bool polar_reaches(double x, double S, double c2, bool cos_nonneg) {
+  const double x2 = x * x, rhs = S * c2;
+  return cos_nonneg ? (x <= 0.0 || x2 <= rhs) : (x < 0.0 && x2 >= rhs);
+}
+
+template <int BITS>
+__device__ __forceinline__ int polar_code(double x, double S, const double *c2) {
+  if (S == 0.0) return 0;  // atan2(0, 0) = 0
+  int lo = 0, hi = (1 << BITS) - 1;
+#pragma unroll
+  for (int it = 0; it < BITS; ++it) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (polar_reaches(x, S, c2[mid], mid <= (1 << (BITS - 1)))) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Azimuth of (a, z) = (x_126, x_127), S = a^2 + z^2.
+template <int BITS>
+__device__ __forceinline__ int azimuth_code(double a, double z, double S, const double *c2) {
+  if (S == 0.0) return 0;
+  constexpr int H = 1 << (BITS - 1), Q = 1 << (BITS - 2);
+  int lo = 0, hi = (1 << BITS) - 1;
+#pragma unroll
+  for (int it = 0; it < BITS; ++it) {
+    const int k = (lo + hi + 1) >> 1;
+    bool reach;
+    if (z >= 0.0) {  // phi in [0, pi]: a <= rho cos(theta_k) for k <= H
+      reach = (k <= H) && polar_reaches(a, S, c2[k], k <= Q);
+    } else {         // phi in (pi, 2 pi): all k <= H; above, a >= rho cos(theta_k)
+      if (k <= H) {
+        reach = true;
+      } else {
+        const double a2 = a * a, rhs = S * c2[k];
+        reach = (k >= 3 * Q) ? (a >= 0.0 && a2 >= rhs) : (a >= 0.0 || a2 <= rhs);
+      }
+    }
+    if (reach) lo = k; else hi = k - 1;
+  }
+  return lo;
+}
+
+template <int BITS>
+__device__ __forceinline__ void lane_codes(const double (&x)[4], const double (&S)[4], double x127, int lane,
+                                           const EncodeSmem &sm, uint8_t *codes) {
+  const double *pc2 = sm.pol_c2 + lut_off(tier_of_bits(BITS));
+  const double *ac2 = sm.az_c2 + lut_off(tier_of_bits(BITS));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int a = 4 * lane + k;
+    int c;
+    if (a < 126) c = polar_code<BITS>(x[k], S[k], pc2);
+    else if (a == 126) c = azimuth_code<BITS>(x[k], x127, S[k], ac2);
+    else c = 0;  // padding field
+    codes[a] = (uint8_t)c;
+  }
+}
+
+// Word w (32 bits) of a slot's bitstream, from the byte-per-angle codes.
+template <int BITS>
+__device__ __forceinline__ uint32_t pack_word(const uint8_t *codes, int w) {
+  const int lo_bit = 32 * w;
+  const int a0 = lo_bit / BITS, a1 = min(127, (lo_bit + 31) / BITS);
+  uint32_t v = 0;
+  for (int a = a0; a <= a1; ++a) {
+    const int sh = a * BITS - lo_bit;
+    const uint32_t c = codes[a];
+    v |= sh >= 0 ? (c << sh) : (c >> (-sh));
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams p) {
+  __shared__ EncodeSmem sm;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  // Edge tables, fp64 (cospi is exact at the multiples of 1/2 that matter).
+  for (int i = tid; i < kLutEntries; i += kEncThreads) {
+    const int t = i < 8 ? 0 : i < 24 ? 1 : i < 88 ? 2 : 3;
+    const int b = bits_of_tier(t), k = i - lut_off(t);
+    const double cp = cospi((double)k / (double)(1 << b));
+    const double ca = cospi((double)k / (double)(1 << (b - 1)));
+    sm.pol_c2[i] = cp * cp;
+    sm.az_c2[i] = ca * ca;
+  }
+  __syncthreads();
+
+  const int64_t nwarps = (int64_t)gridDim.x * kEncWarps;
+  for (int64_t item = (int64_t)blockIdx.x * kEncWarps + wid; item < p.items; item += nwarps) {
+    const int h = (int)(item % p.Hkv);
+    const int64_t bn = item / p.Hkv;
+    const int b = (int)(bn / p.n_new);
+    const int n = (int)(bn % p.n_new);
+    const int pos = p.start_pos[b] + n;
+    if (pos < 0 || pos >= p.max_pages * kPage) {
+      if (lane == 0) set_err(p.err, SPKV_DEVERR_CTX);
+      continue;
+    }
+    const int pid = p.block_table[(int64_t)b * p.max_pages + pos / kPage];
+    if (pid < 0 || pid >= p.num_pages) {
+      if (lane == 0) set_err(p.err, SPKV_DEVERR_PAGE_ID);
+      continue;
+    }
+    const spkv_page_hdr hd = p.hdr[pid];
+    const int bits = hd.bits;
+    if (tier_of_bits(bits) < 0) {
+      if (lane == 0) set_err(p.err, SPKV_DEVERR_BITS);
+      continue;
+    }
+    const uint64_t rec = (uint64_t)hd.code_off16 * 16u + (uint64_t)h * rec_bytes(bits);
+    if (rec + rec_bytes(bits) > p.arena_bytes) {
+      if (lane == 0) set_err(p.err, SPKV_DEVERR_RECORD);
+      continue;
+    }
+    const int slot = pos % kPage;
+
+    // ---- load x (4 per lane) and square in fp64 (exact for bf16 inputs)
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p.keys + item * kD + 4 * lane);
+    double x[4] = {bf16_to_f64(raw.x & 0xffffu), bf16_to_f64(raw.x >> 16), bf16_to_f64(raw.y & 0xffffu),
+                   bf16_to_f64(raw.y >> 16)};
+    // suffix sums S_i = sum_{j >= i} x_j^2: within the lane, then across lanes
+    double S[4];
+    S[3] = x[3] * x[3];
+    S[2] = x[2] * x[2] + S[3];
+    S[1] = x[1] * x[1] + S[2];
+    S[0] = x[0] * x[0] + S[1];
+    double incl = S[0];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double v = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += v;
+    }
+    double after = __shfl_down_sync(0xffffffffu, incl, 1);
+    if (lane == 31) after = 0.0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) S[k] += after;
+    const double x127 = __shfl_sync(0xffffffffu, x[3], 31);
+
+    // ---- angle codes (fp64 decisions), one byte per angle in shared memory
+    uint8_t *codes = sm.codes[wid];
+    switch (bits) {
+      case 3: lane_codes<3>(x, S, x127, lane, sm, codes); break;
+      case 4: lane_codes<4>(x, S, x127, lane, sm, codes); break;
+      case 6: lane_codes<6>(x, S, x127, lane, sm, codes); break;
+      default: lane_codes<8>(x, S, x127, lane, sm, codes); break;
+    }
+    __syncwarp();
+
+    // ---- pack: lane w < 4b builds word w; store chunk-major
+    uint8_t *recp = p.arena + rec;
+    if (lane < 4 * bits) {
+      uint32_t word;
+      switch (bits) {
+        case 3: word = pack_word<3>(codes, lane); break;
+        case 4: word = pack_word<4>(codes, lane); break;
+        case 6: word = pack_word<6>(codes, lane); break;
+        default: word = pack_word<8>(codes, lane); break;
+      }
+      const int chunk = lane >> 2, wic = lane & 3;
+      *reinterpret_cast<uint32_t *>(recp + (chunk * 16 + slot) * 16 + wic * 4) = word;
+    }
+    // ---- radius code (lane 0 holds S_0 = ||k||^2)
+    if (lane == 0) {
+      const float Lf = p.rad_lo[h], Df = p.rad_step[h];
+      int c = 0;
+      if (!(Df > 0.0f) || !isfinite(Df) || !isfinite(Lf)) {
+        set_err(p.err, SPKV_DEVERR_RADIUS);
+      } else if (S[0] > 0.0) {
+        const double t = (log2(sqrt(S[0])) - (double)Lf) / (double)Df + 0.5;
+        c = t <= 0.0 ? 0 : t >= 255.0 ? 255 : (int)floor(t);
+      }
+      recp[256 * bits + slot] = (uint8_t)c;
+    }
+    // ---- value row (optional)
+    if (p.values) {
+      const uint2 v = *reinterpret_cast<const uint2 *>(p.values + item * kD + 4 * lane);
+      uint16_t *dst = p.v_pages + (((int64_t)pid * p.Hkv + h) * kPage + slot) * kD + 4 * lane;
+      *reinterpret_cast<uint2 *>(dst) = v;
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+// Checks shared by every entry point that reads an spkv_cache.
+spkv_status check_cache(const spkv_cache *c) {
+  if (!c) return SPKV_ERR_INVALID_ARG;
+  if (c->head_dim != kD || c->page_size != kPage) return SPKV_ERR_UNSUPPORTED;
+  if (c->num_kv_heads < 1 || c->num_pages < 0) return SPKV_ERR_INVALID_ARG;
+  if (!c->code_arena || !c->hdr || !c->rad_lo_log2 || !c->rad_step_log2 || !c->v_pages)
+    return SPKV_ERR_INVALID_ARG;
+  if (((uintptr_t)c->code_arena & 15) || ((uintptr_t)c->v_pages & 15) || ((uintptr_t)c->hdr & 7))
+    return SPKV_ERR_INVALID_ARG;
+  return SPKV_OK;
+}
+
+int device_sm_count();
+
+}  // namespace spkv
+
+extern "C" spkv_status spkv_encode_keys(const spkv_cache *cache, const uint16_t *keys, const uint16_t *values,
+                                        const int32_t *start_pos, int32_t B, int32_t n_new,
+                                        const int32_t *block_table, int32_t max_pages, void *stream) {
+  using namespace spkv;
+  spkv_status st = check_cache(cache);
+  if (st != SPKV_OK) return st;
+  if (B < 0 || n_new < 0 || max_pages < 0) return SPKV_ERR_INVALID_ARG;
+  if (B == 0 || n_new == 0) return SPKV_OK;
+  if (!keys || !start_pos || !block_table || max_pages == 0) return SPKV_ERR_INVALID_ARG;
+  if (((uintptr_t)keys & 7) || ((uintptr_t)values & 7)) return SPKV_ERR_INVALID_ARG;
+  EncodeParams p;
+  p.arena = cache->code_arena;
+  p.arena_bytes = cache->code_arena_bytes;
+  p.hdr = cache->hdr;
+  p.rad_lo = cache->rad_lo_log2;
+  p.rad_step = cache->rad_step_log2;
+  p.v_pages = cache->v_pages;
+  p.err = cache->err_flags;
+  p.Hkv = cache->num_kv_heads;
+  p.num_pages = cache->num_pages;
+  p.keys = keys;
+  p.values = values;
+  p.start_pos = start_pos;
+  p.block_table = block_table;
+  p.B = B;
+  p.n_new = n_new;
+  p.max_pages = max_pages;
+  p.items = (int64_t)B * n_new * cache->num_kv_heads;
+  const int sms = device_sm_count();
+  if (sms <= 0) return SPKV_ERR_CUDA;
+  const int64_t want = (p.items + kEncWarps - 1) / kEncWarps;
+  const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+  encode_kernel<<<grid, kEncThreads, 0, (cudaStream_t)stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
+}

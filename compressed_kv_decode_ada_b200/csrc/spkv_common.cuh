@@ -1,0 +1,204 @@
+// spkv_common.cuh -- device helpers shared by the libspkv kernels (sm_100a).
+//
+// Method: "SPHERICAL KV: Angle-Domain Attention and Rate-Distortion Retention
+// for Efficient Long-Context Inference", technical summary section 2.1
+// (Angle-Domain Attention), 2.2 (tier-homogeneous pages) and 2.3 (paged,
+// ragged KV substrate).  Layouts and numerical readings: include/spkv.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "spkv.h"
+
+namespace spkv {
+
+constexpr int kD = 128;       // head dimension
+constexpr int kPage = 16;     // tokens per page
+constexpr int kMaxB = 2048;   // largest batch the split kernels accept (2 CTAs / SM for every G)
+constexpr int kTiers = 4;     // b in {3, 4, 6, 8}
+constexpr float kLog2e = 1.4426950408889634f;
+
+__host__ __device__ constexpr int tier_of_bits(int b) { return b == 3 ? 0 : b == 4 ? 1 : b == 6 ? 2 : b == 8 ? 3 : -1; }
+__host__ __device__ constexpr int bits_of_tier(int t) { return t == 0 ? 3 : t == 1 ? 4 : t == 2 ? 6 : 8; }
+// Offset of tier t's 2^b-entry table inside a concatenated {3,4,6,8} table (344 entries).
+__host__ __device__ constexpr int lut_off(int t) { return t == 0 ? 0 : t == 1 ? 8 : t == 2 ? 24 : 88; }
+constexpr int kLutEntries = 344;
+__host__ __device__ constexpr uint32_t rec_bytes(int b) { return 256u * (uint32_t)b + 16u; }
+
+// ------------------------------------------------------------ small helpers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ double bf16_to_f64(uint32_t h16) {
+  double x = (double)__uint_as_float(h16 << 16);
+  return x == 0.0 ? 0.0 : x;  // -0 -> +0
+}
+
+// d = a * b + c on a pair of fp32 lanes (one f32x2 instruction on sm_100a).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void set_err(uint32_t *err, uint32_t bits) {
+  if (err) atomicOr(err, bits);
+}
+
+// ------------------------------------------------------------ mbarrier / bulk copy
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of *bar to complete, giving up after ~1 s of wall
+// time (or as soon as *abort is set by another warp).  On a timeout it sets
+// SPKV_DEVERR_TIMEOUT and *abort, and returns false; callers then carry on
+// with the same control flow (so every barrier is still reached) but the
+// results of this call are flagged as invalid.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                  uint32_t *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if ((it & 63u) == 63u && globaltimer_ns() - t0 > 1000000000ull) {
+      *abort = 1;
+      set_err(err, SPKV_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// 1-D bulk copy global -> this CTA's shared memory; completion is counted in
+// bytes on *bar.  Both addresses 16-byte aligned, bytes a multiple of 16.
+// (No cluster multicast anywhere in this library.)
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ------------------------------------------------------------ work partition
+// The (page, kv head) units of a batch are numbered u = P[b] + h * np_b + j
+// (sequence-major, then kv head, then page), where np_b = ceil(ctx_b / 16)
+// and P is the exclusive prefix sum of np_b * H_kv.  Split c of C owns the
+// contiguous units [floor(c W / C), floor((c+1) W / C)), W = P[B]; each
+// (split, kv-head row bh) intersection is a segment whose partial result goes
+// to workspace slot c + bh (unique because both indices only grow along the
+// unit order).
+
+__device__ __forceinline__ int64_t split_begin(int64_t W, int C, int c) { return (W * (int64_t)c) / C; }
+
+// Pages of a sequence, validated against max_ctx and max_pages.
+__device__ __forceinline__ int seq_pages(int ctx, int max_ctx, int max_pages, uint32_t *err) {
+  if (ctx < 0 || ctx > max_ctx || ctx > max_pages * kPage) {
+    if (ctx != 0) set_err(err, SPKV_DEVERR_CTX);
+    return 0;
+  }
+  return (ctx + kPage - 1) / kPage;
+}
+
+// Block-wide exclusive prefix of np_b * Hkv into P[0..B] (P[B] = W), computed
+// by all `nthreads` threads of the block (a multiple of 32, <= 1024).
+__device__ __forceinline__ void build_prefix(const int32_t *ctx_lens, int B, int Hkv, int max_ctx, int max_pages,
+                                             uint32_t *err, int32_t *P, int32_t *scratch32, int tid,
+                                             int nthreads) {
+  const int per = (B + nthreads - 1) / nthreads;
+  const int b0 = tid * per;
+  int32_t local = 0;
+  for (int i = 0; i < per; ++i) {
+    const int b = b0 + i;
+    if (b < B) {
+      const int np = seq_pages(ctx_lens[b], max_ctx, max_pages, err);
+      P[b] = np * Hkv;  // temporarily the count
+      local += np * Hkv;
+    }
+  }
+  // exclusive scan of `local` across the block
+  const int lane = tid & 31, wid = tid >> 5, nw = nthreads >> 5;
+  int32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) scratch32[wid] = incl;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t run = 0;
+    for (int w = 0; w < nw; ++w) {
+      int32_t v = scratch32[w];
+      scratch32[w] = run;
+      run += v;
+    }
+    scratch32[nw] = run;
+  }
+  __syncthreads();
+  int32_t run = scratch32[wid] + incl - local;
+  for (int i = 0; i < per; ++i) {
+    const int b = b0 + i;
+    if (b < B) {
+      const int32_t cnt = P[b];
+      P[b] = run;
+      run += cnt;
+    }
+  }
+  if (tid == 0) P[B] = scratch32[nw];
+  __syncthreads();
+}
+
+// Largest b with P[b] <= u (P non-decreasing, P[0] = 0, u < P[B]).
+__device__ __forceinline__ int find_seq(const int32_t *P, int B, int64_t u) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)P[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+}  // namespace spkv

@@ -1,0 +1,156 @@
+"""Python entry points with the C ABI's names; argument marshalling only.
+
+Each function checks shapes/dtypes/devices of torch tensors, then calls the
+entry point of libspkv.so of the same name on the current CUDA stream.  All
+arithmetic of the decode path happens in the CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import check, lib
+from .cache import HEAD_DIM, SpkvCache
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, name, dims=None):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dims is not None and t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dims, got {tuple(t.shape)}")
+
+
+def default_splits(B: int, num_kv_heads: int, max_ctx: int) -> int:
+    return int(lib.spkv_decode_default_splits(B, num_kv_heads, max_ctx))
+
+
+def workspace_bytes(B: int, num_q_heads: int, num_kv_heads: int, max_ctx: int, num_splits: int = 0) -> int:
+    return int(lib.spkv_decode_workspace_bytes(B, num_q_heads, num_kv_heads, max_ctx, num_splits))
+
+
+def alloc_workspace(B, num_q_heads, num_kv_heads, max_ctx, num_splits=0, device="cuda") -> torch.Tensor:
+    n = workspace_bytes(B, num_q_heads, num_kv_heads, max_ctx, num_splits)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def encode_keys(cache: SpkvCache, keys: torch.Tensor, start_pos: torch.Tensor, block_table: torch.Tensor,
+                values: torch.Tensor | None = None, stream=None) -> None:
+    """spkv_encode_keys: keys/values [B, n_new, H_kv, 128] bf16 -> page slots."""
+    _need(keys, torch.bfloat16, "keys", 4)
+    B, n_new, hkv, d = keys.shape
+    if hkv != cache.num_kv_heads or d != HEAD_DIM:
+        raise ValueError("keys must be [B, n_new, H_kv, 128]")
+    if values is not None:
+        _need(values, torch.bfloat16, "values", 4)
+        if values.shape != keys.shape:
+            raise ValueError("values must match keys")
+    _need(start_pos, torch.int32, "start_pos", 1)
+    _need(block_table, torch.int32, "block_table", 2)
+    if start_pos.shape[0] != B or block_table.shape[0] != B:
+        raise ValueError("start_pos / block_table batch mismatch")
+    c = cache.c_struct()
+    check(lib.spkv_encode_keys(ctypes.byref(c), _ptr(keys), _ptr(values), _ptr(start_pos), B, n_new,
+                               _ptr(block_table), block_table.shape[1], _stream(stream)), "spkv_encode_keys")
+
+
+def _out_buffer(out, B, Hq, out_dtype, device):
+    if out is None:
+        out = torch.empty((B, Hq, HEAD_DIM), dtype=out_dtype, device=device)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out must be float32 or bfloat16")
+    _need(out, out.dtype, "out", 3)
+    return out
+
+
+def _batch_checks(q, block_table, ctx_lens):
+    _need(q, torch.bfloat16, "q", 3)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(ctx_lens, torch.int32, "ctx_lens", 1)
+    B = q.shape[0]
+    if block_table.shape[0] != B or ctx_lens.shape[0] != B:
+        raise ValueError("batch mismatch between q, block_table and ctx_lens")
+    if q.shape[2] != HEAD_DIM:
+        raise ValueError("q must be [B, Hq, 128]")
+
+
+def _ws(ws, B, Hq, Hkv, max_ctx, num_splits, device):
+    need = workspace_bytes(B, Hq, Hkv, max_ctx, num_splits)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    return ws, ws.numel() * ws.element_size()
+
+
+def decode_attention(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tensor, ctx_lens: torch.Tensor,
+                     max_ctx: int, out=None, out_dtype=torch.float32, ws=None, num_splits: int = 0,
+                     stream=None) -> torch.Tensor:
+    """spkv_decode_attention: ADA decode straight from the codes; returns out [B, Hq, 128]."""
+    _batch_checks(q, block_table, ctx_lens)
+    B, Hq, _ = q.shape
+    out = _out_buffer(out, B, Hq, out_dtype, q.device)
+    ws, wsb = _ws(ws, B, Hq, cache.num_kv_heads, max_ctx, num_splits, q.device)
+    c = cache.c_struct()
+    check(lib.spkv_decode_attention(ctypes.byref(c), _ptr(q), B, Hq, _ptr(block_table), block_table.shape[1],
+                                    _ptr(ctx_lens), int(max_ctx), _ptr(out), int(out.dtype == torch.bfloat16),
+                                    _ptr(ws), wsb, int(num_splits), _stream(stream)), "spkv_decode_attention")
+    return out
+
+
+def dense_decode(k_pages: torch.Tensor, v_pages: torch.Tensor, q: torch.Tensor, block_table: torch.Tensor,
+                 ctx_lens: torch.Tensor, max_ctx: int, keep_mask=None, err=None, out=None,
+                 out_dtype=torch.float32, ws=None, num_splits: int = 0, stream=None) -> torch.Tensor:
+    """spkv_dense_decode: the uncompressed bf16 paged decode (comparison path)."""
+    _need(k_pages, torch.bfloat16, "k_pages", 4)
+    _need(v_pages, torch.bfloat16, "v_pages", 4)
+    _batch_checks(q, block_table, ctx_lens)
+    num_pages, hkv = k_pages.shape[0], k_pages.shape[1]
+    B, Hq, _ = q.shape
+    out = _out_buffer(out, B, Hq, out_dtype, q.device)
+    ws, wsb = _ws(ws, B, Hq, hkv, max_ctx, num_splits, q.device)
+    check(lib.spkv_dense_decode(_ptr(k_pages), _ptr(v_pages), num_pages, hkv, _ptr(keep_mask), _ptr(err), _ptr(q),
+                                B, Hq, _ptr(block_table), block_table.shape[1], _ptr(ctx_lens), int(max_ctx),
+                                _ptr(out), int(out.dtype == torch.bfloat16), _ptr(ws), wsb, int(num_splits),
+                                _stream(stream)), "spkv_dense_decode")
+    return out
+
+
+def decompress_then_dot(cache: SpkvCache, k_scratch: torch.Tensor, q: torch.Tensor, block_table: torch.Tensor,
+                        ctx_lens: torch.Tensor, max_ctx: int, out=None, out_dtype=torch.float32, ws=None,
+                        num_splits: int = 0, stream=None) -> torch.Tensor:
+    """spkv_decompress_then_dot: materialise k~ into k_scratch, then dense decode."""
+    _need(k_scratch, torch.bfloat16, "k_scratch", 4)
+    _batch_checks(q, block_table, ctx_lens)
+    B, Hq, _ = q.shape
+    out = _out_buffer(out, B, Hq, out_dtype, q.device)
+    ws, wsb = _ws(ws, B, Hq, cache.num_kv_heads, max_ctx, num_splits, q.device)
+    c = cache.c_struct()
+    check(lib.spkv_decompress_then_dot(ctypes.byref(c), _ptr(k_scratch), _ptr(q), B, Hq, _ptr(block_table),
+                                       block_table.shape[1], _ptr(ctx_lens), int(max_ctx), _ptr(out),
+                                       int(out.dtype == torch.bfloat16), _ptr(ws), wsb, int(num_splits),
+                                       _stream(stream)), "spkv_decompress_then_dot")
+    return out
+
+
+def debug_logits(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tensor, ctx_lens: torch.Tensor,
+                 max_ctx: int, stream=None) -> torch.Tensor:
+    """spkv_debug_logits: ADA logits [B, Hq, max_ctx] fp32 (NaN where not written)."""
+    _batch_checks(q, block_table, ctx_lens)
+    B, Hq, _ = q.shape
+    logits = torch.full((B, Hq, max(max_ctx, 1)), float("nan"), dtype=torch.float32, device=q.device)
+    c = cache.c_struct()
+    check(lib.spkv_debug_logits(ctypes.byref(c), _ptr(q), B, Hq, _ptr(block_table), block_table.shape[1],
+                                _ptr(ctx_lens), int(max_ctx), _ptr(logits), _stream(stream)), "spkv_debug_logits")
+    return logits

@@ -1,0 +1,194 @@
+/*
+ * spkv.h -- C ABI of libspkv.so: Spherical KV angle-domain attention (ADA)
+ * paged decode for NVIDIA B200 (sm_100a).
+ *
+ * Source of the method ("the pages"): "SPHERICAL KV: Angle-Domain Attention
+ * and Rate-Distortion Retention for Efficient Long-Context Inference",
+ * technical summary, section 2.1 "Angle-Domain Attention (ADA)" (spherical
+ * parametrisation r = ||k||, phi = Phi(k^); logit ~= ||q|| r~ f_b(c_q, c_k);
+ * f_b a fused cosine from angle codes; no dense key ever written to HBM),
+ * section 2.2 (tier-homogeneous pages read by header-guided streaming; the
+ * retention decision z_i and tier b_i) and section 2.3 (dense keys are mapped
+ * to spherical codes and stored in a paged, ragged KV substrate).
+ *
+ * Numerical definitions (readings of the pages, numbered as in the oracle):
+ *   d = 128; angles phi_1..phi_126 in [0, pi], phi_127 in [0, 2 pi) (n-sphere
+ *   chart); b-bit uniform codes c = floor(phi 2^b / range), midpoint
+ *   reconstruction; the query is coded at each page's b; radius code
+ *   c_r = clamp(floor((log2 ||k|| - L_h)/Delta_h + 1/2), 0, 255) with
+ *   r~ = 2^(L_h + c_r Delta_h); logit = ||q|| r~ f_b / sqrt(d); softmax over
+ *   retained slots (an empty set gives 0); out = sum p v over bf16 values.
+ *
+ * ---------------------------------------------------------------- layout
+ * Page size 16 tokens.  All buffers are caller-owned DEVICE memory (except the
+ * spkv_cache struct itself, which is read on the host) and must be 16-byte
+ * aligned.  bf16 values are passed as uint16_t bit patterns.
+ *
+ *   code arena: for page p, hdr[p].code_off16 * 16 is the byte offset of the
+ *   page's block of H_kv records, one per kv head, each
+ *   REC(b) = 256*b + 16 bytes long:
+ *     bytes [0, 256 b):   angle codes of the 16 slots, chunk-major: the 16-byte
+ *                         chunk k (k < b) of slot s sits at (k*16 + s)*16.
+ *                         Concatenating chunks 0..b-1 of a slot gives its
+ *                         128*b-bit little-endian bitstream; angle i
+ *                         (1-based, i <= 127) occupies bits [(i-1) b, i b);
+ *                         the 128th field is padding and is written as 0.
+ *     bytes [256 b, 256 b + 16): radius code of slot s at byte 256 b + s.
+ *   values:  v_pages[p][h][s][0..127] bf16, i.e. [num_pages, H_kv, 16, 128].
+ *   keep mask (optional): keep_mask[p * H_kv + h], bit s = slot s retained.
+ *   block table: block_table[b * max_pages + j] = physical page of the j-th
+ *   16-token page of sequence b; only j < ceil(ctx_len_b / 16) is read.
+ *
+ * ---------------------------------------------------------------- rules
+ * Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ * default stream), never synchronises, and allocates no device memory.
+ * Host-side argument checks run before any launch and return a status; no
+ * C++ exception crosses the ABI.  Device-side problems found while running
+ * (a page id outside [0, num_pages), a header with b not in {3,4,6,8}, a
+ * record beyond the arena, a context length beyond max_ctx) set bits in
+ * *err_flags (if err_flags != NULL) with atomicOr and the offending page or
+ * token is skipped; kernels never trap.
+ */
+#ifndef SPKV_H_
+#define SPKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPKV_API __attribute__((visibility("default")))
+#else
+#define SPKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPKV_OK = 0,
+    SPKV_ERR_INVALID_ARG = 1, /* NULL pointer, negative size, misalignment     */
+    SPKV_ERR_UNSUPPORTED = 2, /* head_dim != 128, page_size != 16, bad G, ...  */
+    SPKV_ERR_WORKSPACE = 3,   /* ws_bytes smaller than the required size        */
+    SPKV_ERR_CUDA = 4         /* a CUDA runtime call or launch failed           */
+} spkv_status;
+
+/* Device error bits written to *err_flags. */
+#define SPKV_DEVERR_PAGE_ID 0x1u   /* block-table entry outside [0, num_pages) */
+#define SPKV_DEVERR_BITS 0x2u      /* page header b not in {3,4,6,8}           */
+#define SPKV_DEVERR_RECORD 0x4u    /* record would lie beyond the code arena   */
+#define SPKV_DEVERR_CTX 0x8u       /* ctx_len < 0 or > max_ctx or > max_pages*16 */
+#define SPKV_DEVERR_TIMEOUT 0x10u  /* a bounded pipeline wait gave up          */
+#define SPKV_DEVERR_RADIUS 0x20u   /* Delta_h <= 0 or not finite               */
+
+/* Per-page header (tier-homogeneous pages, section 2.2): every slot and every
+ * kv head of a page shares one bit width. */
+typedef struct {
+    uint32_t code_off16; /* byte offset of the page's records / 16          */
+    uint8_t bits;        /* b in {3, 4, 6, 8}                                */
+    uint8_t pad[3];
+} spkv_page_hdr;
+
+/* Compressed paged key store plus bf16 value pages.  The struct lives in host
+ * memory; every pointer in it is device memory. */
+typedef struct {
+    int32_t num_kv_heads;        /* H_kv >= 1                                    */
+    int32_t head_dim;            /* must be 128                                  */
+    int32_t page_size;           /* must be 16                                   */
+    int32_t num_pages;           /* physical pages                               */
+    uint8_t *code_arena;         /* records, see layout above                    */
+    uint64_t code_arena_bytes;   /* arena size, for bounds checks                */
+    const spkv_page_hdr *hdr;    /* [num_pages]                                  */
+    const float *rad_lo_log2;    /* [H_kv] L_h                                   */
+    const float *rad_step_log2;  /* [H_kv] Delta_h (> 0)                         */
+    uint16_t *v_pages;           /* [num_pages, H_kv, 16, 128] bf16              */
+    const uint16_t *keep_mask;   /* [num_pages, H_kv] or NULL (all retained)     */
+    uint32_t *err_flags;         /* device word for SPKV_DEVERR_* bits, or NULL  */
+} spkv_cache;
+
+/* Human-readable name of a status. */
+SPKV_API const char *spkv_status_string(spkv_status s);
+
+/* Encode and append keys (and optionally values) into the paged store
+ * (sections 2.1 and 2.3: dense keys -> radius code + packed angle codes).
+ *   keys      [B, n_new, H_kv, 128] bf16, device
+ *   values    [B, n_new, H_kv, 128] bf16, device, or NULL to leave V untouched
+ *   start_pos [B] int32, device: token n of sequence b goes to position
+ *             start_pos[b] + n, i.e. page block_table[b][pos/16], slot pos%16
+ *   block_table [B, max_pages] int32, device
+ * Each key's bit width is its page's hdr.bits.  Angle and radius codes are
+ * decided in fp64 from the exact squares of the bf16 inputs.  Only the slots
+ * written are touched (their code bits, radius byte and, with values, V row).
+ * Positions at or beyond max_pages*16 set SPKV_DEVERR_CTX and are skipped. */
+SPKV_API spkv_status spkv_encode_keys(const spkv_cache *cache, const uint16_t *keys, const uint16_t *values,
+                             const int32_t *start_pos, int32_t B, int32_t n_new,
+                             const int32_t *block_table, int32_t max_pages, void *stream);
+
+/* Number of work partitions ("splits") the decode calls use when num_splits
+ * is 0: a multiple of the device's SM count, at most one per 8 (page, kv
+ * head) units of the largest possible batch.  -1 on a CUDA error. */
+SPKV_API int32_t spkv_decode_default_splits(int32_t B, int32_t num_kv_heads, int32_t max_ctx);
+
+/* Workspace bytes needed by spkv_decode_attention / spkv_dense_decode /
+ * spkv_decompress_then_dot for these sizes and this split count (0 = default).
+ * Returns 0 for invalid sizes. */
+SPKV_API size_t spkv_decode_workspace_bytes(int32_t B, int32_t num_q_heads, int32_t num_kv_heads,
+                                   int32_t max_ctx, int32_t num_splits);
+
+/* ADA decode attention (section 2.1): for every sequence b and query head
+ * hq (kv head h = hq / G, G = Hq / H_kv), over the slots t < ctx_lens[b] that
+ * the keep mask retains:
+ *   logit_t = ||q|| r~_t f_b(c_q, c_t) / sqrt(128),  out = softmax(logit) . V
+ * computed straight from the codes (no dense key is ever written).
+ *   q        [B, Hq, 128] bf16, device
+ *   block_table [B, max_pages] int32, device; ctx_lens [B] int32, device
+ *   max_ctx  host upper bound of ctx_lens (sizes the work); ctx_lens[b]
+ *            larger than max_ctx or than max_pages*16 sets SPKV_DEVERR_CTX
+ *            and that sequence's output is 0
+ *   out      [B, Hq, 128], fp32 (out_is_bf16 = 0) or bf16 (out_is_bf16 = 1)
+ *   ws       device workspace of ws_bytes >= spkv_decode_workspace_bytes(...)
+ *   num_splits  0 = default; otherwise the number of balanced partitions of
+ *            the (page, kv head) work (any value gives the same result up to
+ *            fp32 rounding order)
+ * Supported: G in {1, 2, 4, 8}, B <= 2048. */
+SPKV_API spkv_status spkv_decode_attention(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t num_q_heads,
+                                  const int32_t *block_table, int32_t max_pages, const int32_t *ctx_lens,
+                                  int32_t max_ctx, void *out, int32_t out_is_bf16, void *ws, size_t ws_bytes,
+                                  int32_t num_splits, void *stream);
+
+/* Dense paged decode over bf16 keys, the uncompressed comparison path
+ * (section 4 of the summary compares against dense KV):
+ * logit = q . k / sqrt(128), same paging, mask, split and output rules as
+ * spkv_decode_attention.
+ *   k_pages, v_pages [num_pages, H_kv, 16, 128] bf16, device
+ *   keep_mask [num_pages, H_kv] or NULL;  err_flags device word or NULL */
+SPKV_API spkv_status spkv_dense_decode(const uint16_t *k_pages, const uint16_t *v_pages, int32_t num_pages,
+                              int32_t num_kv_heads, const uint16_t *keep_mask, uint32_t *err_flags,
+                              const uint16_t *q, int32_t B, int32_t num_q_heads, const int32_t *block_table,
+                              int32_t max_pages, const int32_t *ctx_lens, int32_t max_ctx, void *out,
+                              int32_t out_is_bf16, void *ws, size_t ws_bytes, int32_t num_splits,
+                              void *stream);
+
+/* The "decompress, then dot" strawman of the summary's problem statement:
+ * first writes k~ = bf16(r~ u~(c)) for every page the block table references
+ * below ctx_lens into k_scratch ([num_pages, H_kv, 16, 128] bf16, device;
+ * other pages are left untouched), then runs spkv_dense_decode on k_scratch
+ * and cache->v_pages with the UNQUANTISED query.  Same arguments and rules as
+ * spkv_decode_attention otherwise. */
+SPKV_API spkv_status spkv_decompress_then_dot(const spkv_cache *cache, uint16_t *k_scratch, const uint16_t *q, int32_t B,
+                                     int32_t num_q_heads, const int32_t *block_table, int32_t max_pages,
+                                     const int32_t *ctx_lens, int32_t max_ctx, void *out, int32_t out_is_bf16,
+                                     void *ws, size_t ws_bytes, int32_t num_splits, void *stream);
+
+/* Test hook: the ADA logits themselves (natural-log units, before softmax),
+ * logits[b, hq, t] for t < ctx_lens[b]; evicted slots get -inf; entries at or
+ * beyond ctx_lens[b] are not written.  logits: [B, Hq, max_ctx] fp32, device. */
+SPKV_API spkv_status spkv_debug_logits(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t num_q_heads,
+                              const int32_t *block_table, int32_t max_pages, const int32_t *ctx_lens,
+                              int32_t max_ctx, float *logits, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPKV_H_ */

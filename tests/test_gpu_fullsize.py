@@ -1,0 +1,55 @@
+"""Parity at the full workload sizes, in the launch configuration the bench
+times (default split count), on (sequence, kv head) groups the oracle can
+compute one by one, plus properties that hold at any size."""
+import numpy as np
+import pytest
+import torch
+
+from tests import helpers
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def spkv():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import compressed_kv_decode_ada_b200 as m
+    from compressed_kv_decode_ada_b200 import synthetic, workload
+
+    return m, synthetic, workload
+
+
+@pytest.mark.parametrize("cfg,groups", [
+    (1, [(0, 0), (7, 7), (3, 5)]),
+    (2, [(0, 0), (0, 6)]),
+    (3, [(0, 0), (31, 7), (17, 3)]),
+    (4, [(0, 0), (15, 7)]),
+])
+def test_full_size_sampled_parity(spkv, cfg, groups):
+    m, synthetic, workload = spkv
+    wl = synthetic.make_workload(cfg, device="cuda")
+    cache = workload.build_cache(wl)
+    wl.extras["code_offset"] = cache.page_code_offset
+    out = m.decode_attention(cache, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx)
+    torch.cuda.synchronize()
+    assert cache.error_flags() == 0
+    assert torch.isfinite(out).all()
+    outn = out.cpu().numpy()
+    err = helpers.max_abs_diff_groups(outn, wl, groups, helpers.oracle_seq)
+    assert err <= OUT_TOL, err
+    # the encoded bytes of the sampled groups are the oracle's codes
+    arena = cache.arena.cpu().numpy()
+    import oracle
+
+    for b, h in groups[:1]:
+        gc, gr, _ = helpers.gpu_codes_for_seq(arena, wl, b, h)
+        oc, orc, apos, rpos = oracle.encode(wl.keys_bits(b, h), wl.token_bits(b), float(wl.rad_lo[h]),
+                                            float(wl.rad_step[h]), positions=True)
+        assert not ((gc != oc) & ~helpers.near_integer(apos)).any()
+        assert not ((gr != orc) & ~helpers.near_integer(rpos)).any()
+    # property at any size: every output row is a convex combination of value rows
+    vmax = wl.values.float().abs().amax().item()
+    assert outn.max() <= vmax + 1e-3 and outn.min() >= -vmax - 1e-3

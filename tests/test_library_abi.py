@@ -1,0 +1,83 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point that
+include/spkv.h declares, and rejects bad arguments on the host before any
+launch (no GPU is touched by these calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "spkv.h")).read()
+    return sorted(set(re.findall(r"SPKV_API\s+[\w\s\*]+?\b(spkv_\w+)\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import compressed_kv_decode_ada_b200 as m
+
+    return m
+
+
+def test_header_declares_the_entry_points(lib):
+    names = _declared()
+    assert set(names) == set(lib._lib.EXPORTS), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for name in _declared():
+        assert hasattr(raw, name), name
+
+
+def test_status_strings(lib):
+    assert lib.lib.spkv_status_string(0) == b"SPKV_OK"
+    assert lib.lib.spkv_status_string(3) == b"SPKV_ERR_WORKSPACE"
+    assert lib.lib.spkv_status_string(99) == b"SPKV_ERR_UNKNOWN"
+
+
+def _fake_cache(m, **over):
+    c = m._lib.SpkvCacheC()
+    c.num_kv_heads, c.head_dim, c.page_size, c.num_pages = 2, 128, 16, 10
+    c.code_arena, c.code_arena_bytes, c.hdr = 0x10000, 1 << 20, 0x20000
+    c.rad_lo_log2, c.rad_step_log2, c.v_pages = 0x30000, 0x40000, 0x50000
+    c.keep_mask, c.err_flags = None, None
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+def _decode(m, c, B=1, Hq=4, ws_bytes=1 << 20, splits=4, q=0x60000):
+    L = m.lib
+    return L.spkv_decode_attention(ctypes.byref(c), q, B, Hq, 0x70000, 8, 0x80000, 128, 0x90000, 0, 0xA0000,
+                                   ws_bytes, splits, None)
+
+
+def test_host_argument_checks(lib):
+    m = lib
+    L = m.lib
+    assert L.spkv_decode_attention(None, 0, 0, 1, 0, 0, 0, 0, 0, 0, 0, 0, 0, None) == 1
+    assert _decode(m, _fake_cache(m, head_dim=64)) == 2
+    assert _decode(m, _fake_cache(m, page_size=32)) == 2
+    assert _decode(m, _fake_cache(m), Hq=6) == 2           # G = 3
+    assert _decode(m, _fake_cache(m), Hq=3) == 1           # Hq not a multiple of H_kv
+    assert _decode(m, _fake_cache(m, code_arena=0x10001)) == 1  # misaligned arena
+    assert _decode(m, _fake_cache(m), q=0x60002) == 1      # misaligned q
+    assert _decode(m, _fake_cache(m), ws_bytes=16) == 3    # workspace too small
+    assert _decode(m, _fake_cache(m), B=5000) == 2         # batch beyond the supported maximum
+    assert _decode(m, _fake_cache(m), B=0) == 0            # empty batch: nothing to do
+    # encode: negative sizes / misaligned keys
+    c = _fake_cache(m)
+    assert L.spkv_encode_keys(ctypes.byref(c), 0x1000, None, 0x2000, -1, 1, 0x3000, 4, None) == 1
+    assert L.spkv_encode_keys(ctypes.byref(c), 0x1004, None, 0x2000, 1, 1, 0x3000, 4, None) == 1
+    assert L.spkv_encode_keys(ctypes.byref(c), 0x1000, None, 0x2000, 0, 1, 0x3000, 4, None) == 0
+
+
+def test_workspace_formula(lib):
+    # (C + B H_kv) partial slots of G x 132 floats
+    assert lib.workspace_bytes(8, 32, 8, 32768, 296) == (296 + 64) * 4 * 132 * 4
+    assert lib.workspace_bytes(2, 8, 8, 100, 5) == (5 + 16) * 1 * 132 * 4
+    assert lib.workspace_bytes(2, 7, 2, 100, 5) == 0  # Hq not a multiple of H_kv
