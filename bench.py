@@ -130,6 +130,8 @@ def run_spkv(args, rank, world, local):
 
     cfg = dict(synthetic.CONFIGS[args.config])
     cfg["seed"] = int(cfg["seed"]) + 1000 * rank  # each rank: its own independent batch
+    if args.B:
+        cfg["B"] = args.B  # smaller batch, for profiler captures only
     wl = synthetic.make_workload(cfg, device=dev)
     cache = workload.build_cache(wl)
     B, Hq, Hkv = wl.B, wl.Hq, wl.Hkv
@@ -379,6 +381,7 @@ def main():
     ap.add_argument("--impl", default="spkv", choices=["spkv", "reference"])
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--B", type=int, default=0, help="override the batch size (profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--compare", type=int, default=1)
     ap.add_argument("--compare-steps", type=int, default=50)

@@ -52,6 +52,7 @@ class SpkvCacheC(ctypes.Structure):
         ("v_pages", ctypes.c_void_p),
         ("keep_mask", ctypes.c_void_p),
         ("err_flags", ctypes.c_void_p),
+        ("tiers", ctypes.c_uint32),
     ]
 
 

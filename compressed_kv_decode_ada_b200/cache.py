@@ -49,6 +49,8 @@ class SpkvCache:
         hdr[:, 0:4] = (off // 16).astype("<u4").view(np.uint8).reshape(num_pages, 4)
         hdr[:, 4] = page_bits.astype(np.uint8)
         self.page_bits = page_bits
+        # bit t set when some page uses tier t (b = 3, 4, 6, 8)
+        self.tiers = int(sum(1 << t for t, b in enumerate(BIT_WIDTHS) if np.any(page_bits == b)))
         self.page_code_offset = off
         self.arena = torch.zeros(max(arena_bytes, 16), dtype=torch.uint8, device=self.device)
         self.arena_bytes = arena_bytes
@@ -76,6 +78,7 @@ class SpkvCache:
         c.v_pages = self.v_pages.data_ptr()
         c.keep_mask = self.keep_mask.data_ptr() if self.keep_mask is not None else None
         c.err_flags = self.err.data_ptr()
+        c.tiers = self.tiers
         return c
 
     def error_flags(self) -> int:

@@ -1,9 +1,38 @@
 // api.cu -- status strings and per-device properties for libspkv.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "spkv.h"
 
 namespace spkv {
+
+// Tensor map of a bf16 value-page array [num_pages, H_kv, 16, 128] seen as a
+// 2-D tensor of rows x 128 columns, with boxes of 16 rows x 64 columns
+// (128 bytes wide) and the 128-byte shared-memory swizzle.  The encoder is
+// obtained from the driver through the runtime (no link against libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool make_value_tensor_map(CUtensorMap *map, const void *v_pages, uint64_t rows) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !f)
+      return false;
+    fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  if (rows == 0 || rows > 0xffffffffull) return false;
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(v_pages), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 // Streaming-multiprocessor count of the current device (cached per device).
 int device_sm_count() {

@@ -42,11 +42,12 @@ namespace spkv {
 
 spkv_status check_cache(const spkv_cache *c);
 int device_sm_count();
+bool make_value_tensor_map(CUtensorMap *map, const void *v_pages, uint64_t rows);
 
 namespace {
 
-constexpr int kNCW = 4;                      // consumer warps
-constexpr int kThreads = (kNCW + 1) * 32;    // + producer warp
+constexpr int kNCWMax = 6;                   // largest consumer-warp count of any path
+constexpr float kRescaleSlack = 8.0f;        // log2 units a running max may lag the true max
 #define kNegInf (-__int_as_float(0x7f800000))
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -66,32 +67,94 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   return d;
 }
 
+// float2 load from a 32-bit shared-window address of a table that is
+// written once before the consumer loop (so the load may move freely).
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
+// Tensor-core helpers for P.V: one m16n8k16 bf16 MMA with fp32 accumulation,
+// and a transposing 4-tile ldmatrix.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t saddr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr));
+}
+// (x, y) -> bf16x2 (x in the low half), round to nearest, and the bf16x2 of
+// the rounding residuals: x ~= hi + lo to about 16 significant bits.
+__device__ __forceinline__ void split_bf16x2(float x, float y, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x - hf.x, y - hf.y);
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// Warp-wide max of a float through an order-preserving integer key and one
+// redux.sync (NaN-free inputs; -inf allowed).
+__device__ __forceinline__ float warp_max(float x) {
+  const int i = __float_as_int(x);
+  const int key = i >= 0 ? i : (i ^ 0x7fffffff);
+  const int r = __reduce_max_sync(0xffffffffu, key);
+  return __int_as_float(r >= 0 ? r : (r ^ 0x7fffffff));
+}
+
 // ----------------------------------------------------------------- layout
 template <bool ADA, int G>
 struct Layout {
-  static constexpr int NST = ADA ? 12 : 8;                    // ring stages (3 or 2 per consumer warp)
-  static constexpr int STAGE = ADA ? (4096 + 2064) : 8192;    // V page + largest record | K + V page
-  static constexpr int REC_OFF = 4096;                        // ADA: record after the V page
-  static constexpr int KV_OFF = 4096;                         // dense: V after the K page
+  // 5 consumer warps take PAIRS of units (ADA: the two pages of a pair that
+  // share a tier b <= 4 share every query load).  The producer warp streams
+  // only the small per-unit data -- the code record (ADA) or the bf16 K page
+  // (dense) -- through a CTA-wide ring of NST stages; each consumer warp
+  // fetches the value pages of its pair itself, into two private slots, when
+  // it starts the pair, so the V loads overlap the logit computation and a
+  // ring stage is released as soon as the logits are done.
+  static constexpr int NCW = 5;
+  static constexpr int THREADS = (NCW + 1) * 32;               // + producer warp
+  static constexpr int NST = ADA ? (G == 8 ? 16 : 20) : (G == 8 ? 13 : 14);
+  // Value pages land through two 2-D TMA boxes (16 rows x 64 bf16, 128-byte
+  // swizzle): box j holds dims 64 j .. 64 j + 63, row t's 16-byte chunk c
+  // sits at chunk c ^ (t & 7), so the transposing ldmatrix reads of 8
+  // consecutive rows hit 8 distinct bank groups.  1024-byte aligned.
+  static constexpr int VSLOT = 4096;
+  static constexpr int XSTAGE = ADA ? 2064 : 4096;             // code record | dense K page
   static constexpr int QT_HALF = ADA ? (64 * G + 4) : 8 * (8 * G + 4);  // floats, +16 B skew
   static constexpr int QT_TIER = 2 * QT_HALF;
   static constexpr int QT_FLOATS = (ADA ? kTiers : 1) * QT_TIER;
-  static constexpr int CMB = 132;                             // m, l, pad, pad, acc[128]
-  static constexpr int CMB_FLOATS = kNCW * G * CMB;
-  static constexpr int UNION_FLOATS = QT_FLOATS > CMB_FLOATS ? QT_FLOATS : CMB_FLOATS;
-  static constexpr int PBUF_FLOATS = kNCW * kPage * G * 2;
+  static constexpr int PBUF_FLOATS = NCW * G * 2 * kPage;      // p[g][32 slots of 2 pages] per warp
+  static constexpr int C2_BYTES = ADA ? 2 * kLutEntries * 8 : 0;   // fp64 edge tables (query coding)
+  static constexpr int PB_BYTES = PBUF_FLOATS * 4;
+  // the edge tables are only read while the query is coded, the p buffers
+  // only while pages are processed: they share one region
+  static constexpr int PBC2_BYTES = PB_BYTES > C2_BYTES ? PB_BYTES : C2_BYTES;
 
-  static constexpr int off_stage = 0;
-  static constexpr int off_lut = off_stage + NST * STAGE;
-  static constexpr int lut_bytes = ADA ? 2 * kLutEntries * 8 : 0;
-  static constexpr int off_union = off_lut + lut_bytes;
-  static constexpr int off_pbuf = off_union + UNION_FLOATS * 4;
-  static constexpr int off_sc = off_pbuf + PBUF_FLOATS * 4;   // G scales + L_h + Delta_h
-  static constexpr int off_bar = off_sc + ((G + 2) * 4 + 15) / 16 * 16;
-  static constexpr int off_meta = off_bar + 2 * NST * 8;
-  static constexpr int off_misc = off_meta + NST * 16;       // abort flag + scan scratch
+  static constexpr int off_v = 0;                                 // NCW x 2 value slots
+  static constexpr int off_x = off_v + NCW * 2 * VSLOT;           // ring stages
+  // float2 single-angle tables: polar at off_lut, azimuth 384 entries later;
+  // off_lut = 64 (mod 128) puts both b = 4 tables (entry 8 on) on 128 bytes
+  static constexpr int off_lut = (off_x + NST * XSTAGE + 127) / 128 * 128 + 64;
+  static constexpr int LAZ_OFF = 384;  // entries
+  static constexpr int lut_bytes = ADA ? (LAZ_OFF + kLutEntries) * 8 : 0;
+  static constexpr int off_qt = off_lut + lut_bytes;
+  static constexpr int off_pbc2 = off_qt + QT_FLOATS * 4;
+  static constexpr int off_sc = off_pbc2 + PBC2_BYTES;            // G scales + L_h + Delta_h
+  static constexpr int off_bar = off_sc + ((G + 2) * 4 + 15) / 16 * 16;  // full, empty, value slots
+  static constexpr int off_meta = off_bar + (2 * NST + 2 * NCW) * 8;
+  static constexpr int off_misc = off_meta + NST * 32;            // abort flag + scan scratch
   static constexpr int off_P = off_misc + 16 + 36 * 4;
-  static size_t bytes(int B) { return (size_t)off_P + (size_t)(B + 1) * 4 + 16; }
+  // + 1024 bytes of slack to align the carve-up base to 1024
+  static constexpr size_t bytes(int B) { return (size_t)off_P + (size_t)(B + 1) * 4 + 16 + 1024; }
+  // two CTAs per SM: 228 KB of shared memory minus 1 KB reserved per CTA
+  static_assert(bytes(kMaxB) <= (228 * 1024 - 2 * 1024) / 2, "two CTAs per SM must fit");
 };
 
 struct SplitParams {
@@ -103,6 +166,7 @@ struct SplitParams {
   const uint16_t *v_pages;
   const uint16_t *keep;
   uint32_t *err;
+  uint32_t tiers;  // tiers the query is coded for (bit t: b = {3,4,6,8}[t])
   int Hkv, num_pages;
   const uint16_t *q;
   int B, Hq;
@@ -119,6 +183,8 @@ struct StageMeta {
   int bits;    // ADA tier bit width
   int ntok;    // valid slots in the page (1..16)
   uint32_t live;  // keep-mask bits restricted to the first ntok slots
+  int vrow;    // first row of the unit's value page in the value tensor map
+  int pad[3];
 };
 
 // ----------------------------------------------------------- ADA pieces
@@ -137,65 +203,35 @@ __device__ __forceinline__ void build_luts(float2 *lpol, float2 *laz, int tid, i
 }
 
 // One warp: the coded query (section 2.1's c_theta^q; the query is coded at
-// each tier's b) -> decoded unit vector per tier, written to
-// qt[tier * QT_TIER + half * QT_HALF + (pair * G + g) * 2 + e] for slot
-// a = 64 half + 2 pair + e.  Angle codes are decided in fp64.  Returns ||q||.
+// each tier's b with the same exact fp64 edge tests as the keys) -> decoded
+// unit vector per tier, written to
+// qt[tier * QT_TIER + half * QT_HALF + (pair * G + g) * 2 + e] for field
+// a = 64 half + 2 pair + e.  Returns ||q||.
 template <int G, int QT_HALF>
-__device__ float ada_qprep_row(const uint16_t *qrow, int g, const float2 *lpol, const float2 *laz, float *qt,
-                               int lane) {
+__device__ float ada_qprep_row(const uint16_t *qrow, int g, const float2 *lpol, const float2 *laz,
+                               const double *pol_c2, const double *az_c2, float *qt, int lane, uint32_t tiers) {
   const uint2 raw = *reinterpret_cast<const uint2 *>(qrow + 4 * lane);
-  const double x[4] = {bf16_to_f64(raw.x & 0xffffu), bf16_to_f64(raw.x >> 16), bf16_to_f64(raw.y & 0xffffu),
-                       bf16_to_f64(raw.y >> 16)};
-  double S[4];
-  S[3] = x[3] * x[3];
-  S[2] = x[2] * x[2] + S[3];
-  S[1] = x[1] * x[1] + S[2];
-  S[0] = x[0] * x[0] + S[1];
-  double incl = S[0];
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double v = __shfl_down_sync(0xffffffffu, incl, o);
-    if (lane + o < 32) incl += v;
-  }
-  double after = __shfl_down_sync(0xffffffffu, incl, 1);
-  if (lane == 31) after = 0.0;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) S[k] += after;
+  double x[4], S[4];
+  lane_suffix_sums(raw, lane, x, S);
   const double x127 = __shfl_sync(0xffffffffu, x[3], 31);
-  const double nextS0 = __shfl_down_sync(0xffffffffu, S[0], 1);
-  double phi[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int a = 4 * lane + k;
-    const double Snext = k < 3 ? S[k + 1] : (lane == 31 ? 0.0 : nextS0);
-    if (a < 126) {
-      phi[k] = atan2(sqrt(Snext), x[k]);
-    } else if (a == 126) {
-      double v = atan2(x127, x[k]);
-      if (v < 0.0) v += 2.0 * 3.14159265358979323846;
-      phi[k] = v;
-    } else {
-      phi[k] = 0.0;
-    }
-  }
   const double qn = sqrt(__shfl_sync(0xffffffffu, S[0], 0));
 #pragma unroll
   for (int ti = 0; ti < kTiers; ++ti) {
-    const int b = bits_of_tier(ti);
-    const int top = (1 << b) - 1;
+    if (!((tiers >> ti) & 1u)) continue;
+    int c[4];
+    switch (ti) {
+      case 0: lane_codes<3>(x, S, x127, lane, pol_c2, az_c2, c); break;
+      case 1: lane_codes<4>(x, S, x127, lane, pol_c2, az_c2, c); break;
+      case 2: lane_codes<6>(x, S, x127, lane, pol_c2, az_c2, c); break;
+      default: lane_codes<8>(x, S, x127, lane, pol_c2, az_c2, c); break;
+    }
     float2 cs[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int a = 4 * lane + k;
-      if (a < 126) {
-        const int c = min(top, (int)floor(phi[k] * (double)(1 << b) / 3.14159265358979323846));
-        cs[k] = lpol[lut_off(ti) + c];
-      } else if (a == 126) {
-        const int c = min(top, (int)floor(phi[k] * (double)(1 << b) / (2.0 * 3.14159265358979323846)));
-        cs[k] = laz[lut_off(ti) + c];
-      } else {
-        cs[k] = make_float2(1.0f, 0.0f);  // padding field: u_127 = product of all sines
-      }
+      if (a < 126) cs[k] = lpol[lut_off(ti) + c[k]];
+      else if (a == 126) cs[k] = laz[lut_off(ti) + c[k]];
+      else cs[k] = make_float2(1.0f, 0.0f);  // padding field: u_127 = product of all sines
     }
     const float pl1 = cs[0].y, pl2 = pl1 * cs[1].y, pl3 = pl2 * cs[2].y, lane_prod = pl3 * cs[3].y;
     float inc = lane_prod;
@@ -217,16 +253,26 @@ __device__ float ada_qprep_row(const uint16_t *qrow, int g, const float2 *lpol, 
   return (float)qn;
 }
 
+// NB bits of a lane's code words starting at bit `bit` (compile-time after unrolling).
+template <int NB, int NW>
+__device__ __forceinline__ uint32_t bits_at(const uint32_t (&W)[NW], int bit) {
+  const int w = bit >> 5, sh = bit & 31;
+  uint32_t v;
+  if (sh + NB <= 32) v = W[w] >> sh;
+  else v = __funnelshift_r(W[w], W[w + 1], sh);
+  return v & ((1u << NB) - 1u);
+}
 template <int BITS>
 __device__ __forceinline__ uint32_t code_at(const uint32_t (&W)[2 * BITS], int a) {
-  const int bit = a * BITS, w = bit >> 5, sh = bit & 31;
-  uint32_t v;
-  if (sh + BITS <= 32) v = W[w] >> sh;
-  else v = __funnelshift_r(W[w], W[w + 1], sh);
-  return v & ((1u << BITS) - 1u);
+  return bits_at<BITS, 2 * BITS>(W, a * BITS);
 }
 
 // f_b for the 16 slots of one record and the G heads (valid on lanes 0..15).
+// Lane (t, half) runs the prefix product over the 64 fields of its half as two
+// independent sub-chains of 32 fields (A = A1 + P1 A2), and the halves are
+// joined with f = A_0 + P_0 A_1 (P_0 the product of the first half's sines).
+// (cos, sin) of a field comes from the tier's 2^b-entry table; for b = 4 the
+// 16 float2 entries fill one 128-byte row, so the gathers are conflict-free.
 template <int BITS, int G, int QT_HALF>
 __device__ __forceinline__ void ada_page_f(const uint8_t *rec, const float *qt, const float2 *lpol,
                                            const float2 *laz, int lane, float (&f)[G]) {
@@ -253,46 +299,214 @@ __device__ __forceinline__ void ada_page_f(const uint8_t *rec, const float *qt, 
     W[5] = half ? Bv.w : Bv.y;
   }
   const float *qh = qt + half * QT_HALF;
-  const float2 *l62 = half ? laz : lpol;
-  float P = 1.0f;
-  float2 acc[G];
+  const float2 *l62 = half ? laz : lpol;  // field 126 of the second half is the azimuth
+  float2 acc[2][G];
+  float Ps[2];
 #pragma unroll
-  for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
+  for (int sc = 0; sc < 2; ++sc) {
+    Ps[sc] = 1.f;
 #pragma unroll
-  for (int a = 0; a < 64; a += 2) {
-    const uint32_t c0 = code_at<BITS>(W, a), c1 = code_at<BITS>(W, a + 1);
-    float2 e0, e1;
-    if (a == 62) {
-      e0 = l62[c0];
-      const float2 t1 = lpol[half ? 0u : c1];
-      e1 = make_float2(half ? 1.0f : t1.x, half ? 0.0f : t1.y);
-    } else {
-      e0 = lpol[c0];
-      e1 = lpol[c1];
+    for (int g = 0; g < G; ++g) acc[sc][g] = make_float2(0.f, 0.f);
+  }
+#pragma unroll
+  for (int pq = 0; pq < 16; ++pq) {
+#pragma unroll
+    for (int sc = 0; sc < 2; ++sc) {
+      const int pp = pq + 16 * sc;  // pair index in this half: fields 2 pp, 2 pp + 1
+      const uint32_t c0 = code_at<BITS>(W, 2 * pp), c1 = code_at<BITS>(W, 2 * pp + 1);
+      float2 e0, e1;
+      if (pp == 31) {
+        e0 = l62[c0];
+        const float2 t1 = lpol[half ? 0u : c1];
+        e1 = make_float2(half ? 1.0f : t1.x, half ? 0.0f : t1.y);  // padding field: (1, 0)
+      } else {
+        e0 = lpol[c0];
+        e1 = lpol[c1];
+      }
+      const float u0 = Ps[sc] * e0.x, tt = Ps[sc] * e0.y;
+      const float2 uu = make_float2(u0, tt * e1.x);
+      Ps[sc] = tt * e1.y;
+      const float *qp = qh + pp * G * 2;
+      if constexpr (G == 1) {
+        acc[sc][0] = ffma2(uu, *reinterpret_cast<const float2 *>(qp), acc[sc][0]);
+      } else {
+#pragma unroll
+        for (int g = 0; g < G; g += 2) {
+          const float4 q4 = *reinterpret_cast<const float4 *>(qp + 2 * g);
+          acc[sc][g] = ffma2(uu, make_float2(q4.x, q4.y), acc[sc][g]);
+          acc[sc][g + 1] = ffma2(uu, make_float2(q4.z, q4.w), acc[sc][g + 1]);
+        }
+      }
     }
-    const float u0 = P * e0.x;
-    P *= e0.y;
-    const float u1 = P * e1.x;
-    P *= e1.y;
-    const float2 uu = make_float2(u0, u1);
-    const float *qp = qh + (a >> 1) * G * 2;
+  }
+  const float P1 = Ps[0], Pt = Ps[0] * Ps[1];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float A = fmaf(P1, acc[1][g].x + acc[1][g].y, acc[0][g].x + acc[0][g].y);
+    const float Bh = __shfl_down_sync(0xffffffffu, A, 16);
+    f[g] = fmaf(Pt, Bh, A);
+  }
+}
+
+// f_b for two records (pages A and B of the same kv row and tier, b <= 4):
+// lane (t, half) runs one chain of 64 fields for slot t of each page, and
+// every query load serves both.  Results valid on lanes 0..15.
+template <int BITS, int G, int QT_HALF>
+__device__ __forceinline__ void ada_2page_f(const uint8_t *recA, const uint8_t *recB, const float *qt,
+                                            const float2 *lpol, const float2 *laz, int lane, float (&fA)[G],
+                                            float (&fB)[G]) {
+  static_assert(BITS == 3 || BITS == 4, "pair path for b <= 4");
+  const int t = lane & 15, half = lane >> 4;
+  uint32_t W[2][2 * BITS];
+#pragma unroll
+  for (int pg = 0; pg < 2; ++pg) {
+    const uint8_t *rec = pg ? recB : recA;
+    if constexpr (BITS == 4) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(rec + ((half * 2 + k) * 16 + t) * 16);
+        W[pg][4 * k + 0] = v.x;
+        W[pg][4 * k + 1] = v.y;
+        W[pg][4 * k + 2] = v.z;
+        W[pg][4 * k + 3] = v.w;
+      }
+    } else {
+      const uint4 A = *reinterpret_cast<const uint4 *>(rec + ((half + 0) * 16 + t) * 16);
+      const uint4 Bv = *reinterpret_cast<const uint4 *>(rec + ((half + 1) * 16 + t) * 16);
+      W[pg][0] = half ? A.z : A.x;
+      W[pg][1] = half ? A.w : A.y;
+      W[pg][2] = half ? Bv.x : A.z;
+      W[pg][3] = half ? Bv.y : A.w;
+      W[pg][4] = half ? Bv.z : Bv.x;
+      W[pg][5] = half ? Bv.w : Bv.y;
+    }
+  }
+  const float *qh = qt + half * QT_HALF;
+  const float2 *l62 = half ? laz : lpol;
+  float2 acc[2][G];
+  float Ps[2] = {1.f, 1.f};
+#pragma unroll
+  for (int pg = 0; pg < 2; ++pg)
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[pg][g] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int pp = 0; pp < 32; ++pp) {
+    float2 uu[2];
+#pragma unroll
+    for (int pg = 0; pg < 2; ++pg) {
+      const uint32_t c0 = code_at<BITS>(W[pg], 2 * pp), c1 = code_at<BITS>(W[pg], 2 * pp + 1);
+      float2 e0, e1;
+      if (pp == 31) {
+        e0 = l62[c0];
+        const float2 t1 = lpol[half ? 0u : c1];
+        e1 = make_float2(half ? 1.0f : t1.x, half ? 0.0f : t1.y);
+      } else {
+        e0 = lpol[c0];
+        e1 = lpol[c1];
+      }
+      const float u0 = Ps[pg] * e0.x, tt = Ps[pg] * e0.y;
+      uu[pg] = make_float2(u0, tt * e1.x);
+      Ps[pg] = tt * e1.y;
+    }
+    const float *qp = qh + pp * G * 2;
     if constexpr (G == 1) {
       const float2 q2 = *reinterpret_cast<const float2 *>(qp);
-      acc[0] = ffma2(uu, q2, acc[0]);
+      acc[0][0] = ffma2(uu[0], q2, acc[0][0]);
+      acc[1][0] = ffma2(uu[1], q2, acc[1][0]);
     } else {
 #pragma unroll
       for (int g = 0; g < G; g += 2) {
         const float4 q4 = *reinterpret_cast<const float4 *>(qp + 2 * g);
-        acc[g] = ffma2(uu, make_float2(q4.x, q4.y), acc[g]);
-        acc[g + 1] = ffma2(uu, make_float2(q4.z, q4.w), acc[g + 1]);
+        const float2 qa = make_float2(q4.x, q4.y), qb = make_float2(q4.z, q4.w);
+        acc[0][g] = ffma2(uu[0], qa, acc[0][g]);
+        acc[0][g + 1] = ffma2(uu[0], qb, acc[0][g + 1]);
+        acc[1][g] = ffma2(uu[1], qa, acc[1][g]);
+        acc[1][g + 1] = ffma2(uu[1], qb, acc[1][g + 1]);
       }
     }
   }
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const float A = acc[g].x + acc[g].y;
-    const float Bh = __shfl_down_sync(0xffffffffu, A, 16);
-    f[g] = fmaf(P, Bh, A);
+    const float Aa = acc[0][g].x + acc[0][g].y, Ab = acc[1][g].x + acc[1][g].y;
+    const float Ba = __shfl_down_sync(0xffffffffu, Aa, 16), Bb = __shfl_down_sync(0xffffffffu, Ab, 16);
+    fA[g] = fmaf(Ps[0], Ba, Aa);
+    fB[g] = fmaf(Ps[1], Bb, Ab);
+  }
+}
+
+// b = 4 version of ada_2page_f with a rolled loop: each iteration decodes the
+// 16 pairs of one 16-byte code chunk (32 fields) of both pages, so the loop
+// body (and the instruction footprint) is half of the unrolled one.  The
+// (cos, sin) table of b = 4 is 16 float2 = one 128-byte row starting at a
+// 128-byte aligned shared address: a field's entry address is
+// ((chunk word >> shift) & 0x78) | table.
+template <int G, int QT_HALF>
+__device__ __forceinline__ void ada_2page_f4(const uint8_t *recA, const uint8_t *recB, const float *qt,
+                                             uint32_t lpol_s, uint32_t laz_s, int lane, float (&fA)[G],
+                                             float (&fB)[G]) {
+  const int t = lane & 15, half = lane >> 4;
+  const float *qh = qt + half * QT_HALF;
+  float2 acc[2][G];
+  float Ps[2] = {1.f, 1.f};
+#pragma unroll
+  for (int pg = 0; pg < 2; ++pg)
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[pg][g] = make_float2(0.f, 0.f);
+#pragma unroll 1
+  for (int it = 0; it < 2; ++it) {
+    const int chunk = half * 2 + it;
+    const uint4 wa = *reinterpret_cast<const uint4 *>(recA + (chunk * 16 + t) * 16);
+    const uint4 wb = *reinterpret_cast<const uint4 *>(recB + (chunk * 16 + t) * 16);
+    const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
+    // the chunk's last pair is (azimuth, padding) in the second half
+    const bool tail = it == 1 && half;
+    const float *qi = qh + it * 16 * G * 2;
+#pragma unroll
+    for (int pq = 0; pq < 16; ++pq) {
+      float2 uu[2];
+#pragma unroll
+      for (int pg = 0; pg < 2; ++pg) {
+        const uint32_t w = pg ? WB[pq >> 2] : WA[pq >> 2];
+        const int sh0 = 8 * (pq & 3), sh1 = sh0 + 4;  // bit offsets of the two fields
+        const uint32_t o0 = (sh0 >= 3 ? (w >> (sh0 - 3)) : (w << (3 - sh0))) & 0x78u;
+        const uint32_t o1 = (w >> (sh1 - 3)) & 0x78u;
+        float2 e0, e1;
+        if (pq == 15) {
+          e0 = lds_f2((tail ? laz_s : lpol_s) | o0);
+          const float2 t1 = lds_f2(lpol_s | o1);
+          e1 = make_float2(tail ? 1.0f : t1.x, tail ? 0.0f : t1.y);
+        } else {
+          e0 = lds_f2(lpol_s | o0);
+          e1 = lds_f2(lpol_s | o1);
+        }
+        const float u0 = Ps[pg] * e0.x, tt = Ps[pg] * e0.y;
+        uu[pg] = make_float2(u0, tt * e1.x);
+        Ps[pg] = tt * e1.y;
+      }
+      const float *qp = qi + pq * G * 2;
+      if constexpr (G == 1) {
+        const float2 q2 = *reinterpret_cast<const float2 *>(qp);
+        acc[0][0] = ffma2(uu[0], q2, acc[0][0]);
+        acc[1][0] = ffma2(uu[1], q2, acc[1][0]);
+      } else {
+#pragma unroll
+        for (int g = 0; g < G; g += 2) {
+          const float4 q4 = *reinterpret_cast<const float4 *>(qp + 2 * g);
+          const float2 qa = make_float2(q4.x, q4.y), qb = make_float2(q4.z, q4.w);
+          acc[0][g] = ffma2(uu[0], qa, acc[0][g]);
+          acc[0][g + 1] = ffma2(uu[0], qb, acc[0][g + 1]);
+          acc[1][g] = ffma2(uu[1], qa, acc[1][g]);
+          acc[1][g + 1] = ffma2(uu[1], qb, acc[1][g + 1]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float Aa = acc[0][g].x + acc[0][g].y, Ab = acc[1][g].x + acc[1][g].y;
+    const float Ba = __shfl_down_sync(0xffffffffu, Aa, 16), Bb = __shfl_down_sync(0xffffffffu, Ab, 16);
+    fA[g] = fmaf(Ps[0], Ba, Aa);
+    fB[g] = fmaf(Ps[1], Bb, Ab);
   }
 }
 
@@ -342,18 +556,31 @@ __device__ __forceinline__ void dense_page_logits(const uint8_t *kpage, const fl
 }
 
 // ------------------------------------------------------ split kernel
+// Workspace: one partial record (m, l, pad, pad, acc[128]) per query head for
+// every (split c, kv-head row bh) segment and consumer warp w, at
+// ws + (((c + bh) * NCW + w) * G + g) * 132 floats (NCW consumer warps of
+// the path); m is in log2 units.
+constexpr int kPartial = 132;
+
 template <bool ADA, int G>
-__global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
+__global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
+    split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap vmap) {
   using Ly = Layout<ADA, G>;
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t *stages = smem + Ly::off_stage;
+  constexpr int NCW = Ly::NCW, NST = Ly::NST;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t *vslot_all = smem + Ly::off_v;
+  uint8_t *xst_all = smem + Ly::off_x;
   float2 *lpol = reinterpret_cast<float2 *>(smem + Ly::off_lut);
-  float2 *laz = lpol + kLutEntries;
-  float *uni = reinterpret_cast<float *>(smem + Ly::off_union);
-  float *pbuf_all = reinterpret_cast<float *>(smem + Ly::off_pbuf);
+  float2 *laz = lpol + Ly::LAZ_OFF;
+  float *qt = reinterpret_cast<float *>(smem + Ly::off_qt);
+  double *pol_c2 = reinterpret_cast<double *>(smem + Ly::off_pbc2);
+  double *az_c2 = pol_c2 + kLutEntries;
+  float *pbuf_all = reinterpret_cast<float *>(smem + Ly::off_pbc2);
   float *sc = reinterpret_cast<float *>(smem + Ly::off_sc);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + Ly::off_bar);
-  uint64_t *empty = full + Ly::NST;
+  uint64_t *empty = full + NST;
+  uint64_t *vbar_all = empty + NST;  // 2 per consumer warp
   StageMeta *meta = reinterpret_cast<StageMeta *>(smem + Ly::off_meta);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Ly::off_misc);
   int32_t *scratch = reinterpret_cast<int32_t *>(smem + Ly::off_misc + 16);
@@ -362,28 +589,30 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int C = gridDim.x, c = blockIdx.x;
 
-  build_prefix(p.ctx_lens, p.B, p.Hkv, p.max_ctx, p.max_pages, p.err, P, scratch, tid, kThreads);
+  build_prefix(p.ctx_lens, p.B, p.Hkv, p.max_ctx, p.max_pages, p.err, P, scratch, tid, Ly::THREADS);
   const int64_t W = P[p.B];
   const int64_t u0 = split_begin(W, C, c), u1 = split_begin(W, C, c + 1);
   if (u0 >= u1) return;  // uniform across the block
 
   if (tid == 0) {
-    for (int s = 0; s < Ly::NST; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    for (int v = 0; v < 2 * NCW; ++v) mbar_init(&vbar_all[v], 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if constexpr (ADA) build_luts(lpol, laz, tid, kThreads);
+  if constexpr (ADA) build_luts(lpol, laz, tid, Ly::THREADS);
   __syncthreads();
 
   const int n_units = (int)(u1 - u0);
 
-  if (wid == kNCW) {
+  if (wid == NCW) {
     // =========================== producer warp ===========================
-    // Metadata of a batch of 32 units is fetched by the 32 lanes in two
-    // dependent rounds (block table, then header / mask), one batch ahead.
+    // Unit k (CTA-relative) goes to stage k % NST.  Metadata of a batch of 32
+    // units is fetched by the 32 lanes in two dependent rounds (block table,
+    // then header / mask), half a batch ahead.
     struct A_ {
       int pid, ntok, h, ok;
     };
@@ -423,20 +652,18 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     };
     A_ an = phaseA(0);
     B_ bn = phaseB(an);
-    int issued_round[Ly::NST];
-#pragma unroll
-    for (int s = 0; s < Ly::NST; ++s) issued_round[s] = -1;
+    int k_last = -1;
     for (int kb = 0; kb < n_units; kb += 32) {
       const A_ ac = an;
       const B_ bc = bn;
-      // finalise this lane's unit
       int valid = 0;
       uint64_t rec_off = 0, v_off = 0;
       uint32_t rec_sz = 0;
       if (ac.ok) {
+        const int ti = tier_of_bits(bc.bits);
         if (ac.pid < 0 || ac.pid >= p.num_pages) {
           set_err(p.err, SPKV_DEVERR_PAGE_ID);
-        } else if (ADA && tier_of_bits(bc.bits) < 0) {
+        } else if (ADA && (ti < 0 || !((p.tiers >> ti) & 1u))) {
           set_err(p.err, SPKV_DEVERR_BITS);
         } else {
           v_off = ((uint64_t)ac.pid * p.Hkv + ac.h) * (kPage * kD);
@@ -456,31 +683,30 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
       for (int i = 0; i < cnt; ++i) {
         if (i == 16) bn = phaseB(an);
         const int k = kb + i;
-        const int s = k % Ly::NST, r = k / Ly::NST;
-        if (r > 0) mbar_wait_bounded(&empty[s], (uint32_t)(r - 1) & 1u, abort_flag, p.err);
+        const int s = k % NST, r = k / NST;
+        if (r > 0) mbar_wait_bounded(&empty[s], (uint32_t)(r - 1) & 1u, abort_flag, p.err, 64);
         if (lane == i) {
           StageMeta m;
           m.valid = valid && !*abort_flag;
           m.bits = bc.bits;
           m.ntok = ac.ntok;
           m.live = live;
+          m.vrow = (int)(v_off / kD);  // (pid * H_kv + h) * 16
           meta[s] = m;
-          uint8_t *st = stages + s * Ly::STAGE;
+          uint8_t *xst = xst_all + s * Ly::XSTAGE;
           if (m.valid) {
             if constexpr (ADA) {
-              mbar_arrive_expect_tx(&full[s], rec_sz + 4096u);
-              bulk_g2s(st, p.v_pages + v_off, 4096u, &full[s]);
-              bulk_g2s(st + Ly::REC_OFF, p.arena + rec_off, rec_sz, &full[s]);
+              mbar_arrive_expect_tx(&full[s], rec_sz);
+              bulk_g2s(xst, p.arena + rec_off, rec_sz, &full[s]);
             } else {
-              mbar_arrive_expect_tx(&full[s], 8192u);
-              bulk_g2s(st, p.k_pages + v_off, 4096u, &full[s]);
-              bulk_g2s(st + Ly::KV_OFF, p.v_pages + v_off, 4096u, &full[s]);
+              mbar_arrive_expect_tx(&full[s], 4096u);
+              bulk_g2s(xst, p.k_pages + v_off, 4096u, &full[s]);
             }
           } else {
             mbar_arrive(&full[s]);
           }
         }
-        issued_round[s] = r;
+        k_last = k;
         __syncwarp();
       }
       if (cnt <= 16) bn = phaseB(an);
@@ -489,17 +715,26 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     // them (bounded) before the CTA's shared memory can be released.
     if (*abort_flag && lane == 0) {
       volatile int dummy = 0;
-      for (int s = 0; s < Ly::NST; ++s)
-        if (issued_round[s] >= 0) mbar_wait_bounded(&full[s], (uint32_t)issued_round[s] & 1u, &dummy, nullptr);
+      for (int s = 0; s < NST; ++s) {
+        const int kk = k_last - ((k_last - s) % NST + NST) % NST;  // last unit in stage s
+        if (kk >= 0) mbar_wait_bounded(&full[s], (uint32_t)(kk / NST) & 1u, &dummy, nullptr);
+      }
     }
     return;
   }
 
   // ============================= consumer warps ============================
-  const int ctid = tid;  // 0 .. 127
-  float *pbuf = pbuf_all + wid * (kPage * G * 2);
+  // Units are grouped in pairs (2i, 2i + 1); pair i belongs to warp i % NCW.
+  // A pair whose two units lie in one segment and share a tier b <= 4 is
+  // decoded in one pass (every query load serves both pages); any other
+  // unit is decoded on its own.
+  float *pbuf = pbuf_all + wid * (G * 2 * kPage);
+  const int grp = lane >> 2, tig = lane & 3;
+  uint8_t *const vslot[2] = {vslot_all + (2 * wid) * Ly::VSLOT, vslot_all + (2 * wid + 1) * Ly::VSLOT};
+  uint64_t *const vbar = vbar_all + 2 * wid;
+  uint32_t vphase[2] = {0u, 0u};
+  int vpending[2] = {-1, -1};  // phase of a value load a failed wait left in flight
   int64_t u = u0;
-  int k = wid;  // next unit index of this warp (CTA-relative)
   while (u < u1) {
     const int b = find_seq(P, p.B, u);
     const int np = (P[b + 1] - P[b]) / p.Hkv;
@@ -508,174 +743,286 @@ __global__ void __launch_bounds__(kThreads) split_kernel(const SplitParams p) {
     const int64_t seg_end = seg_hi < u1 ? seg_hi : u1;
     const int bh = b * p.Hkv + h;
 
-    // ---- per-segment query preparation
-    for (int g = wid; g < G; g += kNCW) {
+    // ---- per-segment query preparation (every consumer warp is past the
+    // previous segment's last page: the edge tables may overwrite the p buffers)
+    named_bar_sync(1, NCW * 32);
+    if constexpr (ADA) build_edge_tables(pol_c2, az_c2, tid, NCW * 32);
+    named_bar_sync(1, NCW * 32);
+    for (int g = wid; g < G; g += NCW) {
       const uint16_t *qrow = p.q + ((int64_t)b * p.Hq + (int64_t)h * G + g) * kD;
       if constexpr (ADA) {
-        const float qn = ada_qprep_row<G, Ly::QT_HALF>(qrow, g, lpol, laz, uni, lane);
+        const float qn = ada_qprep_row<G, Ly::QT_HALF>(qrow, g, lpol, laz, pol_c2, az_c2, qt, lane, p.tiers);
         if (lane == 0) sc[g] = qn * kLog2e * 0.08838834764831845f;
       } else {
-        dense_qprep_row<G, Ly::QT_HALF>(qrow, g, uni, lane);
+        dense_qprep_row<G, Ly::QT_HALF>(qrow, g, qt, lane);
       }
     }
     if constexpr (ADA) {
-      if (ctid == 0) {
+      if (tid == 0) {
         sc[G] = p.rad_lo[h];
         sc[G + 1] = p.rad_step[h];
       }
     }
-    named_bar_sync(1, kNCW * 32);
+    named_bar_sync(1, NCW * 32);
 
     float m[G], lsum[G];
-    float2 acc[G][2];
+    // P.V accumulators in m16n8k16 fragment layout (D^T = V^T P^T):
+    // d[mb][0..1] = dim 16 mb + grp, heads 2 tig, 2 tig + 1; d[mb][2..3] = dim + 8
+    float d[8][4];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       m[g] = kNegInf;
       lsum[g] = 0.f;
-      acc[g][0] = acc[g][1] = make_float2(0.f, 0.f);
     }
+#pragma unroll
+    for (int mb = 0; mb < 8; ++mb) d[mb][0] = d[mb][1] = d[mb][2] = d[mb][3] = 0.f;
     float scg[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) scg[g] = sc[g];
     const float Lh = ADA ? sc[G] : 0.f, Dh = ADA ? sc[G + 1] : 0.f;
 
-    for (; u0 + k < seg_end; k += kNCW) {
-      const int s = k % Ly::NST, r = k / Ly::NST;
-      const bool ok = mbar_wait_bounded(&full[s], (uint32_t)r & 1u, abort_flag, p.err);
-      const StageMeta mt = meta[s];
-      const uint8_t *st = stages + s * Ly::STAGE;
-      if (ok && mt.valid && mt.live) {
-        float l2[G];
-        if constexpr (ADA) {
-          float f[G];
-          const int ti = tier_of_bits(mt.bits);
-          const float *qt = uni + ti * Ly::QT_TIER;
-          const float2 *lp = lpol + lut_off(ti), *la = laz + lut_off(ti);
-          const uint8_t *rec = st + Ly::REC_OFF;
-          switch (mt.bits) {
-            case 3: ada_page_f<3, G, Ly::QT_HALF>(rec, qt, lp, la, lane, f); break;
-            case 4: ada_page_f<4, G, Ly::QT_HALF>(rec, qt, lp, la, lane, f); break;
-            case 6: ada_page_f<6, G, Ly::QT_HALF>(rec, qt, lp, la, lane, f); break;
-            default: ada_page_f<8, G, Ly::QT_HALF>(rec, qt, lp, la, lane, f); break;
-          }
-          const float rc = (float)rec[256 * mt.bits + (lane & 15)];
-          const float rad = fast_exp2(fmaf(rc, Dh, Lh));
-#pragma unroll
-          for (int g = 0; g < G; ++g) l2[g] = scg[g] * rad * f[g];
-        } else {
-          dense_page_logits<G, Ly::QT_HALF>(st, uni, lane, l2);
+    // logits of a page (ADA from codes, dense from bf16 keys), lanes 0..15
+    auto page_logits = [&](const StageMeta &mt, const uint8_t *xst, float (&l2)[G]) {
+      if constexpr (ADA) {
+        float f[G];
+        const int ti = tier_of_bits(mt.bits);
+        const float *q0 = qt + ti * Ly::QT_TIER;
+        const float2 *lp = lpol + lut_off(ti), *la = laz + lut_off(ti);
+        switch (mt.bits) {
+          case 3: ada_page_f<3, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
+          case 4: ada_page_f<4, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
+          case 6: ada_page_f<6, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
+          default: ada_page_f<8, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
         }
-        const bool alive = lane < 16 && ((mt.live >> (lane & 15)) & 1u);
-        float pg[G];
+        const float rad = fast_exp2(fmaf((float)xst[256 * mt.bits + (lane & 15)], Dh, Lh));
+#pragma unroll
+        for (int g = 0; g < G; ++g) l2[g] = scg[g] * rad * f[g];
+      } else {
+        dense_page_logits<G, Ly::QT_HALF>(xst, qt, lane, l2);
+      }
+    };
+
+    // online softmax over the pages of a pair (slots 0..15 and 16..31 of
+    // pbuf; use[q] = 0 drops page q) followed by P.V on tensor cores.  The
+    // running max m only moves when a page's max exceeds it by more than
+    // kRescaleSlack, so p <= 2^8 and the accumulators are rescaled on few pages.
+    auto softmax_pv = [&](const bool (&use)[2], const StageMeta (&mt)[2], const float (&l2)[2][G],
+                          uint8_t *const (&vs)[2]) {
+      float x[2][G];
+      bool alive[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        alive[q] = use[q] && lane < 16 && ((mt[q].live >> (lane & 15)) & 1u);
+#pragma unroll
+        for (int g = 0; g < G; ++g) x[q][g] = alive[q] ? l2[q][g] : kNegInf;
+      }
+      bool moved = false;
+      float alpha[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float mx = warp_max(fmaxf(x[0][g], x[1][g]));
+        alpha[g] = 1.f;
+        if (mx > m[g] + kRescaleSlack) {  // warp-uniform
+          alpha[g] = m[g] == kNegInf ? 0.f : fast_exp2(m[g] - mx);
+          m[g] = mx;
+          moved = true;
+        }
+        const float pa = (alive[0] && m[g] != kNegInf) ? fast_exp2(x[0][g] - m[g]) : 0.f;
+        const float pb = (alive[1] && m[g] != kNegInf) ? fast_exp2(x[1][g] - m[g]) : 0.f;
+        lsum[g] = fmaf(lsum[g], alpha[g], pa + pb);
+        if (lane < 16) {
+          pbuf[g * 2 * kPage + lane] = pa;
+          pbuf[g * 2 * kPage + kPage + lane] = pb;
+        }
+      }
+      if (moved) {  // rescale the fragments of heads 2 tig, 2 tig + 1
+        float a0 = 1.f, a1 = 1.f;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          float x = alive ? l2[g] : kNegInf;
-          float mx = x;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          const float mnew = fmaxf(m[g], mx);
-          const float alpha = mnew == kNegInf ? 1.f : fast_exp2(m[g] - mnew);
-          pg[g] = alive ? fast_exp2(x - mnew) : 0.f;
-          lsum[g] = fmaf(lsum[g], alpha, pg[g]);
-          const float2 a2 = make_float2(alpha, alpha);
-          acc[g][0] = fmul2(acc[g][0], a2);
-          acc[g][1] = fmul2(acc[g][1], a2);
-          m[g] = mnew;
+          if (2 * tig == g) a0 = alpha[g];
+          if (2 * tig + 1 == g) a1 = alpha[g];
         }
-        if (lane < 16) {
-          float *dst = pbuf + lane * G * 2;
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            dst[2 * g] = pg[g];
-            dst[2 * g + 1] = pg[g];
-          }
-        }
-        __syncwarp();
-        const uint8_t *vpage = ADA ? st : st + Ly::KV_OFF;
-#pragma unroll
-        for (int t = 0; t < kPage; ++t) {
-          if ((mt.live >> t) & 1u) {
-            const uint2 vw = *reinterpret_cast<const uint2 *>(vpage + t * 256 + lane * 8);
-            const float2 v01 = make_float2(bf16lo(vw.x), bf16hi(vw.x));
-            const float2 v23 = make_float2(bf16lo(vw.y), bf16hi(vw.y));
-            const float *pp = pbuf + t * G * 2;
-            if constexpr (G == 1) {
-              const float2 p2 = *reinterpret_cast<const float2 *>(pp);
-              acc[0][0] = ffma2(p2, v01, acc[0][0]);
-              acc[0][1] = ffma2(p2, v23, acc[0][1]);
-            } else {
-#pragma unroll
-              for (int g = 0; g < G; g += 2) {
-                const float4 p4 = *reinterpret_cast<const float4 *>(pp + 2 * g);
-                const float2 pa = make_float2(p4.x, p4.y), pb = make_float2(p4.z, p4.w);
-                acc[g][0] = ffma2(pa, v01, acc[g][0]);
-                acc[g][1] = ffma2(pa, v23, acc[g][1]);
-                acc[g + 1][0] = ffma2(pb, v01, acc[g + 1][0]);
-                acc[g + 1][1] = ffma2(pb, v23, acc[g + 1][1]);
-              }
-            }
-          }
+        for (int mb = 0; mb < 8; ++mb) {
+          d[mb][0] *= a0;
+          d[mb][1] *= a1;
+          d[mb][2] *= a0;
+          d[mb][3] *= a1;
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (!use[q]) continue;  // warp-uniform
+        // rows past the context end (last page) may hold anything: zero them
+        // so that p = 0 times the row stays 0
+        if (mt[q].ntok < kPage) {
+          for (int i = lane; i < (kPage - mt[q].ntok) * 16; i += 32) {
+            const int row = mt[q].ntok + (i >> 4), box = (i >> 3) & 1, ch = i & 7;
+            *reinterpret_cast<uint4 *>(vs[q] + box * 2048 + row * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        // B = P^T (16 slots x heads) as bf16 hi + lo
+        uint32_t bh0 = 0u, bh1 = 0u, bl0 = 0u, bl1 = 0u;
+        if (grp < G) {
+          const float *pr = pbuf + grp * 2 * kPage + q * kPage;
+          const float2 pa = *reinterpret_cast<const float2 *>(pr + 2 * tig);
+          const float2 pb = *reinterpret_cast<const float2 *>(pr + 2 * tig + 8);
+          split_bf16x2(pa.x, pa.y, bh0, bl0);
+          split_bf16x2(pb.x, pb.y, bh1, bl1);
+        }
+        const int vt = (lane & 7) + 8 * (lane >> 4);  // value row (slot) this lane addresses
+        const uint32_t vrow = smem_u32(vs[q]) + (uint32_t)(vt * 128);
+        const uint32_t jsel = (lane >> 3) & 1u, t7 = (uint32_t)(vt & 7);
+#pragma unroll
+        for (int mb = 0; mb < 8; ++mb) {
+          uint32_t a[4];
+          const uint32_t j = 2u * (uint32_t)(mb & 3) + jsel;  // 16-byte chunk within the box row
+          ldsm_x4_trans(a, vrow + (uint32_t)(mb >> 2) * 2048u + ((j ^ t7) << 4));
+          mma_bf16_16816(d[mb], a, bh0, bh1);
+          mma_bf16_16816(d[mb], a, bl0, bl1);
+        }
+      }
+    };
+
+    // ---- this segment's units: CTA-relative [ks, ke)
+    const int ks = (int)(u - u0), ke = (int)(seg_end - u0);
+    int i = ks >> 1;
+    i += ((wid - i) % NCW + NCW) % NCW;
+    for (; 2 * i < ke; i += NCW) {
+      const int ka = 2 * i < ks ? ks : 2 * i;
+      const int kz = 2 * i + 2 > ke ? ke : 2 * i + 2;  // units [ka, kz) of pair i in this segment
+      const int n = kz - ka;
+      StageMeta mt[2];
+      const uint8_t *xst[2];
+      bool use[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        use[q] = false;
+        xst[q] = xst_all;
+        mt[q] = StageMeta{};
+        if (q < n) {
+          const int k = ka + q, s = k % NST;
+          const bool ok = mbar_wait_bounded(&full[s], (uint32_t)(k / NST) & 1u, abort_flag, p.err);
+          mt[q] = meta[s];
+          use[q] = ok && mt[q].valid && mt[q].live;
+          xst[q] = xst_all + s * Ly::XSTAGE;
+        }
+      }
+      // the pair's value pages, into this warp's slots (overlaps the logits)
+      if (lane == 0) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          if (use[q]) {
+            uint64_t *vb = &vbar[q];
+            mbar_arrive_expect_tx(vb, 4096u);
+            tma_load_2d(vslot[q], &vmap, 0, mt[q].vrow, vb);
+            tma_load_2d(vslot[q] + 2048, &vmap, 64, mt[q].vrow, vb);
+          }
+        }
+      }
+      float l2[2][G];
+      bool paired = false;
+      if constexpr (ADA) {
+        paired = use[0] && use[1] && mt[0].bits == mt[1].bits && mt[0].bits <= 4;
+      }
+      if (paired) {
+        if constexpr (ADA) {
+          float fa[G], fb[G];
+          const int ti = tier_of_bits(mt[0].bits);
+          const float *q0 = qt + ti * Ly::QT_TIER;
+          const float2 *lp = lpol + lut_off(ti), *la = laz + lut_off(ti);
+          if (mt[0].bits == 4)
+            ada_2page_f4<G, Ly::QT_HALF>(xst[0], xst[1], q0, smem_u32(lp), smem_u32(la), lane, fa, fb);
+          else
+            ada_2page_f<3, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb);
+          const int bits = mt[0].bits;
+          const float ra = fast_exp2(fmaf((float)xst[0][256 * bits + (lane & 15)], Dh, Lh));
+          const float rb = fast_exp2(fmaf((float)xst[1][256 * bits + (lane & 15)], Dh, Lh));
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            l2[0][g] = scg[g] * ra * fa[g];
+            l2[1][g] = scg[g] * rb * fb[g];
+          }
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          if (use[q]) page_logits(mt[q], xst[q], l2[q]);  // warp-uniform
+        }
+      }
+      // the ring stages are free once the logits are known
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&empty[ka % NST]);
+        if (n == 2) mbar_arrive(&empty[(ka + 1) % NST]);
+      }
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (use[q]) {
+          if (!mbar_wait_bounded(&vbar[q], vphase[q], abort_flag, p.err)) vpending[q] = (int)vphase[q];
+          vphase[q] ^= 1u;
+        }
+      }
+      softmax_pv(use, mt, l2, vslot);
+      __syncwarp();
     }
 
-    // ---- merge the 4 warps' states of this segment into one partial
+    // ---- this warp's partial of the segment, straight to the workspace
 #pragma unroll
     for (int g = 0; g < G; ++g) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) lsum[g] += __shfl_xor_sync(0xffffffffu, lsum[g], o);
     }
-    named_bar_sync(1, kNCW * 32);  // every warp is done with the query table
-    float *cmb = uni + wid * G * Ly::CMB;
+    float *part = p.ws + ((int64_t)(c + bh) * NCW + wid) * G * kPartial;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float *cg = cmb + g * Ly::CMB;
-      if (lane == 0) {
-        cg[0] = m[g];
-        cg[1] = lsum[g];
-      }
-      *reinterpret_cast<float4 *>(cg + 4 + 4 * lane) = make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
+      if (lane == 0) *reinterpret_cast<float2 *>(part + g * kPartial) = make_float2(m[g], lsum[g]);
     }
-    named_bar_sync(1, kNCW * 32);
-    float *slot = p.ws + (int64_t)(c + bh) * G * Ly::CMB;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float mw[kNCW], M = kNegInf;
+    for (int j = 0; j < 2; ++j) {
+      const int g = 2 * tig + j;
+      if (g < G) {
+        float *pg = part + g * kPartial + 4;
 #pragma unroll
-      for (int w = 0; w < kNCW; ++w) {
-        mw[w] = uni[(w * G + g) * Ly::CMB];
-        M = fmaxf(M, mw[w]);
-      }
-      float num = 0.f, den = 0.f;
-#pragma unroll
-      for (int w = 0; w < kNCW; ++w) {
-        const float s = mw[w] == kNegInf ? 0.f : fast_exp2(mw[w] - M);
-        num = fmaf(s, uni[(w * G + g) * Ly::CMB + 4 + ctid], num);
-        den = fmaf(s, uni[(w * G + g) * Ly::CMB + 1], den);
-      }
-      slot[g * Ly::CMB + 4 + ctid] = num;
-      if (ctid == 0) {
-        slot[g * Ly::CMB + 0] = M;
-        slot[g * Ly::CMB + 1] = den;
+        for (int mb = 0; mb < 8; ++mb) {
+          pg[16 * mb + grp] = d[mb][j];
+          pg[16 * mb + grp + 8] = d[mb][2 + j];
+        }
       }
     }
-    named_bar_sync(1, kNCW * 32);  // the union region is reused by the next query table
     u = seg_end;
+  }
+  // After an abort a value load of this warp may still be landing in its
+  // slots: wait for it (bounded) before the shared memory is released.
+  if (lane == 0) {
+    volatile int dummy = 0;
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      if (vpending[q] >= 0) mbar_wait_bounded(&vbar[q], (uint32_t)vpending[q], &dummy, nullptr);
   }
 }
 
 // ------------------------------------------------------------ merge kernel
-// One block per (sequence, kv head): combine the partials of the splits that
-// covered its units, for its G query heads.  out = sum_s 2^(m_s - M) acc_s /
-// sum_s 2^(m_s - M) l_s, or 0 when no slot was retained.
+// One block per (sequence, query head): combine the partials of every
+// (split, consumer warp) that covered the head's kv row.
+//   out = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s   (0 when nothing
+// was retained).  The partials' (m, l) are loaded in parallel into shared
+// memory, then each thread sums its dimension over all partials.
 template <int G>
-__global__ void __launch_bounds__(128) merge_kernel(const float *ws, int C, const int32_t *ctx_lens, int B, int Hkv,
-                                                    int Hq, int max_ctx, int max_pages, void *out, int out_bf16) {
-  constexpr int CMB = 132;
+__global__ void __launch_bounds__(128) merge_kernel(const float *ws, int C, int NCW, const int32_t *ctx_lens, int B,
+                                                    int Hkv, int Hq, int max_ctx, int max_pages, void *out,
+                                                    int out_bf16) {
+  constexpr int kChunk = 256;  // partials per pass
   __shared__ int64_t red[2][4];
-  const int bh = blockIdx.x, b = bh / Hkv, h = bh % Hkv;
+  __shared__ float wgt[kChunk];
+  __shared__ float lsh[kChunk];
+  __shared__ int64_t off[kChunk];
+  __shared__ float Msh;
+  const int hq = blockIdx.x % Hq, b = blockIdx.x / Hq;
+  const int h = hq / G, g = hq % G, bh = b * Hkv + h;
   const int tid = threadIdx.x;
   int64_t before = 0, total = 0;
   for (int i = tid; i < B; i += 128) {
@@ -696,41 +1043,75 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, int C, cons
   before = red[0][0] + red[0][1] + red[0][2] + red[0][3];
   const int64_t W = red[1][0] + red[1][1] + red[1][2] + red[1][3];
   const int np = seq_pages(ctx_lens[b], max_ctx, max_pages, nullptr);
-  const int64_t a = before + (int64_t)h * np, e = a + np;
-  float res[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) res[g] = 0.f;
+  float num = 0.f, den = 0.f;
   if (np > 0) {
+    const int64_t a = before + (int64_t)h * np, e = a + np;
     const int64_t cf = ((a + 1) * C + W - 1) / W - 1;
     int64_t cl = (e * C + W - 1) / W - 1;
     if (cl > C - 1) cl = C - 1;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float M = kNegInf;
-      for (int64_t cc = cf; cc <= cl; ++cc) {
-        if (split_begin(W, C, (int)cc) >= split_begin(W, C, (int)cc + 1)) continue;
-        M = fmaxf(M, ws[((cc + bh) * G + g) * CMB]);
-      }
-      float num = 0.f, den = 0.f;
-      if (M != kNegInf) {
-        for (int64_t cc = cf; cc <= cl; ++cc) {
-          if (split_begin(W, C, (int)cc) >= split_begin(W, C, (int)cc + 1)) continue;
-          const float *sl = ws + ((cc + bh) * G + g) * CMB;
-          const float mm = sl[0];
-          const float s = mm == kNegInf ? 0.f : fast_exp2(mm - M);
-          num = fmaf(s, sl[4 + tid], num);
-          den = fmaf(s, sl[1], den);
+    const int64_t nparts = (cl - cf + 1) * NCW;
+    float M = kNegInf;
+    // pass 1: the running max over all partials
+    for (int64_t base = 0; base < nparts; base += kChunk) {
+      for (int i = tid; i < kChunk; i += 128) {
+        float mm = kNegInf;
+        if (base + i < nparts) {
+          const int64_t cc = cf + (base + i) / NCW;
+          const int w = (int)((base + i) % NCW);
+          if (split_begin(W, C, (int)cc) < split_begin(W, C, (int)cc + 1))
+            mm = ws[(((cc + bh) * NCW + w) * G + g) * kPartial];
         }
+        wgt[i] = mm;
       }
-      res[g] = den > 0.f ? num / den : 0.f;
+      __syncthreads();
+      if (tid == 0) {
+        for (int i = 0; i < kChunk && base + i < nparts; ++i) M = fmaxf(M, wgt[i]);
+      }
+      __syncthreads();
+    }
+    if (tid == 0) Msh = M;
+    __syncthreads();
+    M = Msh;
+    if (M != kNegInf) {
+      for (int64_t base = 0; base < nparts; base += kChunk) {
+        for (int i = tid; i < kChunk; i += 128) {
+          float wv = 0.f, lv = 0.f;
+          int64_t o = -1;
+          if (base + i < nparts) {
+            const int64_t cc = cf + (base + i) / NCW;
+            const int w = (int)((base + i) % NCW);
+            if (split_begin(W, C, (int)cc) < split_begin(W, C, (int)cc + 1)) {
+              o = (((cc + bh) * NCW + w) * G + g) * kPartial;
+              const float mm = ws[o];
+              if (mm != kNegInf) {
+                wv = fast_exp2(mm - M);
+                lv = ws[o + 1];
+              } else {
+                o = -1;
+              }
+            }
+          }
+          wgt[i] = wv;
+          lsh[i] = lv;
+          off[i] = o;
+        }
+        __syncthreads();
+        const int n = (int)min((int64_t)kChunk, nparts - base);
+#pragma unroll 8
+        for (int i = 0; i < n; ++i) {
+          if (off[i] >= 0) {
+            num = fmaf(wgt[i], ws[off[i] + 4 + tid], num);
+            den = fmaf(wgt[i], lsh[i], den);
+          }
+        }
+        __syncthreads();
+      }
     }
   }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const int64_t o = ((int64_t)b * Hq + (int64_t)h * G + g) * kD + tid;
-    if (out_bf16) reinterpret_cast<__nv_bfloat16 *>(out)[o] = __float2bfloat16_rn(res[g]);
-    else reinterpret_cast<float *>(out)[o] = res[g];
-  }
+  const float res = den > 0.f ? num / den : 0.f;
+  const int64_t o = ((int64_t)b * Hq + hq) * kD + tid;
+  if (out_bf16) reinterpret_cast<__nv_bfloat16 *>(out)[o] = __float2bfloat16_rn(res);
+  else reinterpret_cast<float *>(out)[o] = res;
 }
 
 // ---------------------------------------------------- decompress kernel
@@ -816,6 +1197,7 @@ template <int G>
 __global__ void __launch_bounds__(32) debug_logits_kernel(SplitParams p, float *logits) {
   constexpr int QT_HALF = 64 * G + 4;
   __shared__ float2 lpol[kLutEntries], laz[kLutEntries];
+  __shared__ double pol_c2[kLutEntries], az_c2[kLutEntries];
   __shared__ __align__(16) float qt[kTiers * 2 * QT_HALF];
   __shared__ __align__(16) uint8_t rec[2064];
   __shared__ float qn[G];
@@ -841,12 +1223,13 @@ __global__ void __launch_bounds__(32) debug_logits_kernel(SplitParams p, float *
     return;
   }
   build_luts(lpol, laz, lane, 32);
+  build_edge_tables(pol_c2, az_c2, lane, 32);
   for (uint32_t i = lane * 16; i < rsz; i += 32 * 16)
     *reinterpret_cast<uint4 *>(rec + i) = *reinterpret_cast<const uint4 *>(p.arena + roff + i);
   __syncwarp();
   for (int g = 0; g < G; ++g) {
     const float n = ada_qprep_row<G, QT_HALF>(p.q + ((int64_t)b * p.Hq + (int64_t)h * G + g) * kD, g, lpol, laz,
-                                              qt, lane);
+                                              pol_c2, az_c2, qt, lane, 0xfu);
     if (lane == 0) qn[g] = n;
   }
   __syncwarp();
@@ -885,7 +1268,8 @@ int blocks_per_sm(size_t smem) {
     configured[dev] = 1;
   }
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<ADA, G>, kThreads, smem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<ADA, G>, Layout<ADA, G>::THREADS, smem) !=
+      cudaSuccess)
     return -1;
   return n;
 }
@@ -938,25 +1322,28 @@ spkv_status launch_split_and_merge(const DecodeArgs &a, cudaStream_t stream) {
   const size_t smem = smem_for<ADA>(a.G, a.sp.B);
   if (blocks_per_sm_for<ADA>(a.G, smem) < 1) return SPKV_ERR_CUDA;
   const int C = a.num_splits;
+  CUtensorMap vmap;
+  if (!make_value_tensor_map(&vmap, a.sp.v_pages, (uint64_t)a.sp.num_pages * a.sp.Hkv * kPage))
+    return a.sp.num_pages == 0 ? SPKV_ERR_INVALID_ARG : SPKV_ERR_CUDA;
   switch (a.G) {
-    case 1: split_kernel<ADA, 1><<<C, kThreads, smem, stream>>>(a.sp); break;
-    case 2: split_kernel<ADA, 2><<<C, kThreads, smem, stream>>>(a.sp); break;
-    case 4: split_kernel<ADA, 4><<<C, kThreads, smem, stream>>>(a.sp); break;
-    case 8: split_kernel<ADA, 8><<<C, kThreads, smem, stream>>>(a.sp); break;
+    case 1: split_kernel<ADA, 1><<<C, Layout<ADA, 1>::THREADS, smem, stream>>>(a.sp, vmap); break;
+    case 2: split_kernel<ADA, 2><<<C, Layout<ADA, 2>::THREADS, smem, stream>>>(a.sp, vmap); break;
+    case 4: split_kernel<ADA, 4><<<C, Layout<ADA, 4>::THREADS, smem, stream>>>(a.sp, vmap); break;
+    case 8: split_kernel<ADA, 8><<<C, Layout<ADA, 8>::THREADS, smem, stream>>>(a.sp, vmap); break;
   }
   if (cudaGetLastError() != cudaSuccess) return SPKV_ERR_CUDA;
-  const int nb = a.sp.B * a.sp.Hkv;
+  const int nb = a.sp.B * a.sp.Hq;
   switch (a.G) {
-    case 1: merge_kernel<1><<<nb, 128, 0, stream>>>(a.sp.ws, C, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
-    case 2: merge_kernel<2><<<nb, 128, 0, stream>>>(a.sp.ws, C, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
-    case 4: merge_kernel<4><<<nb, 128, 0, stream>>>(a.sp.ws, C, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
-    case 8: merge_kernel<8><<<nb, 128, 0, stream>>>(a.sp.ws, C, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
+    case 1: merge_kernel<1><<<nb, 128, 0, stream>>>(a.sp.ws, C, Layout<ADA, 1>::NCW, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
+    case 2: merge_kernel<2><<<nb, 128, 0, stream>>>(a.sp.ws, C, Layout<ADA, 2>::NCW, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
+    case 4: merge_kernel<4><<<nb, 128, 0, stream>>>(a.sp.ws, C, Layout<ADA, 4>::NCW, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
+    case 8: merge_kernel<8><<<nb, 128, 0, stream>>>(a.sp.ws, C, Layout<ADA, 8>::NCW, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
   }
   return cudaGetLastError() == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
 }
 
 size_t ws_bytes_for(int B, int Hq, int Hkv, int C) {
-  return (size_t)(C + B * Hkv) * (size_t)(Hq / Hkv) * 132u * sizeof(float);
+  return (size_t)(C + B * Hkv) * kNCWMax * (size_t)(Hq / Hkv) * kPartial * sizeof(float);
 }
 
 // Shared validation of the batch arguments; fills sp's batch fields.
@@ -997,6 +1384,7 @@ void fill_cache(SplitParams &sp, const spkv_cache *c) {
   sp.v_pages = c->v_pages;
   sp.keep = c->keep_mask;
   sp.err = c->err_flags;
+  sp.tiers = c->tiers ? c->tiers : 0xfu;
   sp.Hkv = c->num_kv_heads;
   sp.num_pages = c->num_pages;
 }

@@ -38,74 +38,11 @@ struct EncodeParams {
   int64_t items;  // B * n_new * Hkv
 };
 
-// Shared tables: squared cosines of the cell edges, per tier.
-//   polar   edge k of b bits: theta = k pi / 2^b          (k in [0, 2^b))
-//   azimuth edge k of b bits: theta = k 2 pi / 2^b        (k in [0, 2^b))
 struct EncodeSmem {
   double pol_c2[kLutEntries];
   double az_c2[kLutEntries];
   uint8_t codes[kEncWarps][128];
 };
-
-// phi >= theta_k for a polar angle, given x = x_i, S = S_i (S > 0), the edge's
-// squared cosine c2 and whether its cosine is non-negative.
-__device__ __forceinline__ bool polar_reaches(double x, double S, double c2, bool cos_nonneg) {
-  const double x2 = x * x, rhs = S * c2;
-  return cos_nonneg ? (x <= 0.0 || x2 <= rhs) : (x < 0.0 && x2 >= rhs);
-}
-
-template <int BITS>
-__device__ __forceinline__ int polar_code(double x, double S, const double *c2) {
-  if (S == 0.0) return 0;  // atan2(0, 0) = 0
-  int lo = 0, hi = (1 << BITS) - 1;
-#pragma unroll
-  for (int it = 0; it < BITS; ++it) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (polar_reaches(x, S, c2[mid], mid <= (1 << (BITS - 1)))) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-// Azimuth of (a, z) = (x_126, x_127), S = a^2 + z^2.
-template <int BITS>
-__device__ __forceinline__ int azimuth_code(double a, double z, double S, const double *c2) {
-  if (S == 0.0) return 0;
-  constexpr int H = 1 << (BITS - 1), Q = 1 << (BITS - 2);
-  int lo = 0, hi = (1 << BITS) - 1;
-#pragma unroll
-  for (int it = 0; it < BITS; ++it) {
-    const int k = (lo + hi + 1) >> 1;
-    bool reach;
-    if (z >= 0.0) {  // phi in [0, pi]: a <= rho cos(theta_k) for k <= H
-      reach = (k <= H) && polar_reaches(a, S, c2[k], k <= Q);
-    } else {         // phi in (pi, 2 pi): all k <= H; above, a >= rho cos(theta_k)
-      if (k <= H) {
-        reach = true;
-      } else {
-        const double a2 = a * a, rhs = S * c2[k];
-        reach = (k >= 3 * Q) ? (a >= 0.0 && a2 >= rhs) : (a >= 0.0 || a2 <= rhs);
-      }
-    }
-    if (reach) lo = k; else hi = k - 1;
-  }
-  return lo;
-}
-
-template <int BITS>
-__device__ __forceinline__ void lane_codes(const double (&x)[4], const double (&S)[4], double x127, int lane,
-                                           const EncodeSmem &sm, uint8_t *codes) {
-  const double *pc2 = sm.pol_c2 + lut_off(tier_of_bits(BITS));
-  const double *ac2 = sm.az_c2 + lut_off(tier_of_bits(BITS));
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int a = 4 * lane + k;
-    int c;
-    if (a < 126) c = polar_code<BITS>(x[k], S[k], pc2);
-    else if (a == 126) c = azimuth_code<BITS>(x[k], x127, S[k], ac2);
-    else c = 0;  // padding field
-    codes[a] = (uint8_t)c;
-  }
-}
 
 // Word w (32 bits) of a slot's bitstream, from the byte-per-angle codes.
 template <int BITS>
@@ -124,15 +61,7 @@ __device__ __forceinline__ uint32_t pack_word(const uint8_t *codes, int w) {
 __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams p) {
   __shared__ EncodeSmem sm;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  // Edge tables, fp64 (cospi is exact at the multiples of 1/2 that matter).
-  for (int i = tid; i < kLutEntries; i += kEncThreads) {
-    const int t = i < 8 ? 0 : i < 24 ? 1 : i < 88 ? 2 : 3;
-    const int b = bits_of_tier(t), k = i - lut_off(t);
-    const double cp = cospi((double)k / (double)(1 << b));
-    const double ca = cospi((double)k / (double)(1 << (b - 1)));
-    sm.pol_c2[i] = cp * cp;
-    sm.az_c2[i] = ca * ca;
-  }
+  build_edge_tables(sm.pol_c2, sm.az_c2, tid, kEncThreads);
   __syncthreads();
 
   const int64_t nwarps = (int64_t)gridDim.x * kEncWarps;
@@ -164,36 +93,23 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams 
     }
     const int slot = pos % kPage;
 
-    // ---- load x (4 per lane) and square in fp64 (exact for bf16 inputs)
+    // ---- load x (4 per lane); exact squares and suffix sums in fp64
     const uint2 raw = *reinterpret_cast<const uint2 *>(p.keys + item * kD + 4 * lane);
-    double x[4] = {bf16_to_f64(raw.x & 0xffffu), bf16_to_f64(raw.x >> 16), bf16_to_f64(raw.y & 0xffffu),
-                   bf16_to_f64(raw.y >> 16)};
-    // suffix sums S_i = sum_{j >= i} x_j^2: within the lane, then across lanes
-    double S[4];
-    S[3] = x[3] * x[3];
-    S[2] = x[2] * x[2] + S[3];
-    S[1] = x[1] * x[1] + S[2];
-    S[0] = x[0] * x[0] + S[1];
-    double incl = S[0];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double v = __shfl_down_sync(0xffffffffu, incl, o);
-      if (lane + o < 32) incl += v;
-    }
-    double after = __shfl_down_sync(0xffffffffu, incl, 1);
-    if (lane == 31) after = 0.0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) S[k] += after;
+    double x[4], S[4];
+    lane_suffix_sums(raw, lane, x, S);
     const double x127 = __shfl_sync(0xffffffffu, x[3], 31);
 
     // ---- angle codes (fp64 decisions), one byte per angle in shared memory
     uint8_t *codes = sm.codes[wid];
+    int c4[4];
     switch (bits) {
-      case 3: lane_codes<3>(x, S, x127, lane, sm, codes); break;
-      case 4: lane_codes<4>(x, S, x127, lane, sm, codes); break;
-      case 6: lane_codes<6>(x, S, x127, lane, sm, codes); break;
-      default: lane_codes<8>(x, S, x127, lane, sm, codes); break;
+      case 3: lane_codes<3>(x, S, x127, lane, sm.pol_c2, sm.az_c2, c4); break;
+      case 4: lane_codes<4>(x, S, x127, lane, sm.pol_c2, sm.az_c2, c4); break;
+      case 6: lane_codes<6>(x, S, x127, lane, sm.pol_c2, sm.az_c2, c4); break;
+      default: lane_codes<8>(x, S, x127, lane, sm.pol_c2, sm.az_c2, c4); break;
     }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) codes[4 * lane + k] = (uint8_t)c4[k];
     __syncwarp();
 
     // ---- pack: lane w < 4b builds word w; store chunk-major

@@ -6,6 +6,7 @@
 // ragged KV substrate).  Layouts and numerical readings: include/spkv.h.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -15,7 +16,7 @@ namespace spkv {
 
 constexpr int kD = 128;       // head dimension
 constexpr int kPage = 16;     // tokens per page
-constexpr int kMaxB = 2048;   // largest batch the split kernels accept (2 CTAs / SM for every G)
+constexpr int kMaxB = 1024;   // largest batch the split kernels accept (2 CTAs / SM for every G)
 constexpr int kTiers = 4;     // b in {3, 4, 6, 8}
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -92,11 +93,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // SPKV_DEVERR_TIMEOUT and *abort, and returns false; callers then carry on
 // with the same control flow (so every barrier is still reached) but the
 // results of this call are flagged as invalid.
+// sleep_ns > 0 backs off between polls (for waiters off the critical path).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                                  uint32_t *err) {
+                                                  uint32_t *err, uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if ((it & 63u) == 63u && globaltimer_ns() - t0 > 1000000000ull) {
@@ -116,6 +119,22 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// 2-D tiled TMA load (box of the tensor map at element coordinates (x, y))
+// into this CTA's shared memory, completion counted on *bar.  No multicast.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA) accesses of the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
@@ -199,6 +218,109 @@ __device__ __forceinline__ int find_seq(const int32_t *P, int B, int64_t u) {
     if ((int64_t)P[mid] <= u) lo = mid; else hi = mid - 1;
   }
   return lo;
+}
+
+// ------------------------------------------------------------ exact code decisions
+// Squared cosines of the cell edges, fp64, for the four tiers concatenated:
+//   polar   edge k of b bits: theta = k pi / 2^b      -> pol_c2[lut_off(t) + k]
+//   azimuth edge k of b bits: theta = k 2 pi / 2^b    -> az_c2[lut_off(t) + k]
+// Computed as (1 + cos 2 theta) / 2 so that the edges at multiples of pi/4,
+// the only ones a bf16 input can hit exactly, get the exact values 1, 1/2, 0:
+// an exact tie is then decided exactly (to the upper cell).
+__device__ __forceinline__ void build_edge_tables(double *pol_c2, double *az_c2, int tid, int nthreads) {
+  for (int i = tid; i < kLutEntries; i += nthreads) {
+    const int t = i < 8 ? 0 : i < 24 ? 1 : i < 88 ? 2 : 3;
+    const int b = bits_of_tier(t), k = i - lut_off(t);
+    pol_c2[i] = 0.5 * (1.0 + cospi((double)(2 * k) / (double)(1 << b)));
+    az_c2[i] = 0.5 * (1.0 + cospi((double)(4 * k) / (double)(1 << b)));
+  }
+}
+
+// phi >= theta_k for a polar angle, given x = x_i, S = S_i = sum_{j>=i} x_j^2
+// (S > 0), the edge's squared cosine c2 and whether its cosine is >= 0:
+// phi >= theta  <=>  cos(phi) = x / sqrt(S) <= cos(theta).
+__device__ __forceinline__ bool polar_reaches(double x, double S, double c2, bool cos_nonneg) {
+  const double x2 = x * x, rhs = S * c2;
+  return cos_nonneg ? (x <= 0.0 || x2 <= rhs) : (x < 0.0 && x2 >= rhs);
+}
+
+// floor(phi 2^b / pi) clamped to 2^b - 1 for phi = atan2(sqrt(S_{i+1}), x_i),
+// by binary search over the edges (the largest edge the angle reaches).
+template <int BITS>
+__device__ __forceinline__ int polar_code(double x, double S, const double *c2) {
+  if (S == 0.0) return 0;  // atan2(0, 0) = 0
+  int lo = 0, hi = (1 << BITS) - 1;
+#pragma unroll
+  for (int it = 0; it < BITS; ++it) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (polar_reaches(x, S, c2[mid], mid <= (1 << (BITS - 1)))) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// floor(phi 2^b / 2 pi) for the azimuth phi = atan2(z, a) taken in [0, 2 pi),
+// with a = x_126, z = x_127, S = a^2 + z^2.  z >= 0: phi in [0, pi] and the
+// polar test applies to the edges k <= 2^(b-1); z < 0: phi in (pi, 2 pi), every
+// edge k <= 2^(b-1) is reached and above it phi >= theta_k <=> a >= rho cos theta_k.
+template <int BITS>
+__device__ __forceinline__ int azimuth_code(double a, double z, double S, const double *c2) {
+  if (S == 0.0) return 0;
+  constexpr int H = 1 << (BITS - 1), Q = 1 << (BITS - 2);
+  int lo = 0, hi = (1 << BITS) - 1;
+#pragma unroll
+  for (int it = 0; it < BITS; ++it) {
+    const int k = (lo + hi + 1) >> 1;
+    bool reach;
+    if (z >= 0.0) {
+      reach = (k <= H) && polar_reaches(a, S, c2[k], k <= Q);
+    } else if (k <= H) {
+      reach = true;
+    } else {
+      const double a2 = a * a, rhs = S * c2[k];
+      reach = (k >= 3 * Q) ? (a >= 0.0 && a2 >= rhs) : (a >= 0.0 || a2 <= rhs);
+    }
+    if (reach) lo = k; else hi = k - 1;
+  }
+  return lo;
+}
+
+// The four fp64 inputs of one warp lane (x_{4l..4l+3}) and the suffix sums
+// S_i = sum_{j >= i} x_j^2 (squares of bf16 values are exact in fp64).
+__device__ __forceinline__ void lane_suffix_sums(uint2 raw, int lane, double (&x)[4], double (&S)[4]) {
+  x[0] = bf16_to_f64(raw.x & 0xffffu);
+  x[1] = bf16_to_f64(raw.x >> 16);
+  x[2] = bf16_to_f64(raw.y & 0xffffu);
+  x[3] = bf16_to_f64(raw.y >> 16);
+  S[3] = x[3] * x[3];
+  S[2] = x[2] * x[2] + S[3];
+  S[1] = x[1] * x[1] + S[2];
+  S[0] = x[0] * x[0] + S[1];
+  double incl = S[0];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double v = __shfl_down_sync(0xffffffffu, incl, o);
+    if (lane + o < 32) incl += v;
+  }
+  double after = __shfl_down_sync(0xffffffffu, incl, 1);
+  if (lane == 31) after = 0.0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) S[k] += after;
+}
+
+// Angle codes of the lane's four fields a = 4 lane + k at b = BITS bits
+// (field 126 is the azimuth, field 127 the zero padding).
+template <int BITS>
+__device__ __forceinline__ void lane_codes(const double (&x)[4], const double (&S)[4], double x127, int lane,
+                                           const double *pol_c2, const double *az_c2, int (&c)[4]) {
+  const double *pc2 = pol_c2 + lut_off(tier_of_bits(BITS));
+  const double *ac2 = az_c2 + lut_off(tier_of_bits(BITS));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int a = 4 * lane + k;
+    if (a < 126) c[k] = polar_code<BITS>(x[k], S[k], pc2);
+    else if (a == 126) c[k] = azimuth_code<BITS>(x[k], x127, S[k], ac2);
+    else c[k] = 0;
+  }
 }
 
 }  // namespace spkv

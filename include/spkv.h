@@ -104,6 +104,9 @@ typedef struct {
     uint16_t *v_pages;           /* [num_pages, H_kv, 16, 128] bf16              */
     const uint16_t *keep_mask;   /* [num_pages, H_kv] or NULL (all retained)     */
     uint32_t *err_flags;         /* device word for SPKV_DEVERR_* bits, or NULL  */
+    uint32_t tiers;              /* bit t set when some page uses b = {3,4,6,8}[t]; 0 = any.
+                                    Decoding codes the query only for these tiers; a page
+                                    of another tier sets SPKV_DEVERR_BITS and is skipped. */
 } spkv_cache;
 
 /* Human-readable name of a status. */
@@ -150,7 +153,7 @@ SPKV_API size_t spkv_decode_workspace_bytes(int32_t B, int32_t num_q_heads, int3
  *   num_splits  0 = default; otherwise the number of balanced partitions of
  *            the (page, kv head) work (any value gives the same result up to
  *            fp32 rounding order)
- * Supported: G in {1, 2, 4, 8}, B <= 2048. */
+ * Supported: G in {1, 2, 4, 8}, B <= 1024. */
 SPKV_API spkv_status spkv_decode_attention(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t num_q_heads,
                                   const int32_t *block_table, int32_t max_pages, const int32_t *ctx_lens,
                                   int32_t max_ctx, void *out, int32_t out_is_bf16, void *ws, size_t ws_bytes,

