@@ -128,7 +128,7 @@ def run_spkv(args, rank, world, local):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    cfg = dict(synthetic.CONFIGS[args.config])
+    cfg = dict(synthetic.WORKLOADS[args.workload])
     cfg["seed"] = int(cfg["seed"]) + 1000 * rank  # each rank: its own independent batch
     if args.B:
         cfg["B"] = args.B  # smaller batch, for profiler captures only
@@ -223,7 +223,7 @@ def run_spkv(args, rank, world, local):
     if rank == 0:
         peak, peak_kind = _peaks()
         achieved = bytes_step / (dec_ms * 1e-3) / 1e9
-        traffic = _committed_traffic(args.config)
+        traffic = _committed_traffic(args.workload)
         h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
         d2h = out_h.numel() * out_h.element_size()
         result = {
@@ -313,7 +313,7 @@ def compare_paths(args, spkv, workload, wl, cache, ctx, max_ctx, splits, ws, str
     return res
 
 
-def _committed_traffic(config):
+def _committed_traffic(workload):
     """ncu DRAM bytes per launch of the ADA split kernel, from the committed
     profile summary, if it was taken on the current kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -324,7 +324,7 @@ def _committed_traffic(config):
         return None
     src = os.path.join(ROOT, "compressed_kv_decode_ada_b200", "csrc", "decode.cu")
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    ent = d.get(str(config))
+    ent = d.get(workload)
     if not ent or ent.get("decode_cu_sha256_16") != sha:
         return None
     return ent.get("dram_bytes_per_step")
@@ -341,7 +341,7 @@ def cpu_oracle(args, budget_s: float):
     import oracle
     from compressed_kv_decode_ada_b200 import synthetic
 
-    cfg = dict(synthetic.CONFIGS[args.config])
+    cfg = dict(synthetic.WORKLOADS[args.workload])
     wl = synthetic.make_workload(cfg, device="cpu", B=min(cfg["B"], 2))
     cores = _cores()
     groups = [(b, h) for b in range(wl.B) for h in range(wl.Hkv)]
@@ -379,7 +379,8 @@ def main():
     ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="spkv", choices=["spkv", "reference"])
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--workload", default="llama3_8b_b8_h32x8_t32768_b4",
+                    help="one of compressed_kv_decode_ada_b200.synthetic.WORKLOADS")
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=500)
@@ -398,12 +399,11 @@ def main():
         cb = cpu_oracle(args, args.cpu_budget)
         from compressed_kv_decode_ada_b200 import synthetic
 
-        wl_cfg = synthetic.CONFIGS[args.config]
         line = {"metric": "ADA decode KV tokens/s on 1 B200; achieved HBM GB/s as % of peak", "impl": "reference",
                 "value": cb["value"], "unit": "KV tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": wl_cfg["name"]}, "cpu_baseline": cb,
+                "config": {"workload": args.workload}, "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "KV tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)

@@ -36,18 +36,22 @@ HEAD_DIM = 128
 PAGE = 16
 ROPE_BASE = 500000.0
 
-# The five workload shapes.  'ctx' is a fixed length or ('loguniform', lo, hi).
-CONFIGS = {
-    0: dict(name="tiny_b1_h1_t4096_b4", B=1, Hq=1, Hkv=1, ctx=4096, rope=False, mixed=False, mask=False, seed=0),
-    1: dict(name="llama3_8b_b8_h32x8_t32768_b4", B=8, Hq=32, Hkv=8, ctx=32768, rope=True, mixed=False, mask=False,
-            seed=1),
-    2: dict(name="long_b1_h32x8_t131072_b4", B=1, Hq=32, Hkv=8, ctx=131072, rope=True, mixed=False, mask=False,
-            seed=2),
-    3: dict(name="ragged_rdr_b32_h32x8_t1k-64k_mixed_b_mask25", B=32, Hq=32, Hkv=8, ctx=("loguniform", 1024, 65536),
-            rope=True, mixed=True, mask=True, seed=3),
-    4: dict(name="70b_b16_h64x8_t16384_b4_encode", B=16, Hq=64, Hkv=8, ctx=16384, rope=True, mixed=False,
-            mask=False, seed=4),
+# The five workload shapes, by name.  'ctx' is a fixed length or
+# ('loguniform', lo, hi).
+TINY = "tiny_b1_h1_t4096_b4"
+LLAMA3_8B = "llama3_8b_b8_h32x8_t32768_b4"
+LONG_128K = "long_b1_h32x8_t131072_b4"
+RAGGED_RDR = "ragged_rdr_b32_h32x8_t1k-64k_mixed_b_mask25"
+SHAPE_70B = "70b_b16_h64x8_t16384_b4_encode"
+WORKLOADS = {
+    TINY: dict(B=1, Hq=1, Hkv=1, ctx=4096, rope=False, mixed=False, mask=False, seed=0),
+    LLAMA3_8B: dict(B=8, Hq=32, Hkv=8, ctx=32768, rope=True, mixed=False, mask=False, seed=1),
+    LONG_128K: dict(B=1, Hq=32, Hkv=8, ctx=131072, rope=True, mixed=False, mask=False, seed=2),
+    RAGGED_RDR: dict(B=32, Hq=32, Hkv=8, ctx=("loguniform", 1024, 65536), rope=True, mixed=True, mask=True, seed=3),
+    SHAPE_70B: dict(B=16, Hq=64, Hkv=8, ctx=16384, rope=True, mixed=False, mask=False, seed=4),
 }
+for _n, _c in WORKLOADS.items():
+    _c["name"] = _n
 
 
 @dataclass
@@ -136,13 +140,13 @@ def _rope_(k: torch.Tensor, pos0: int) -> None:
     k[..., half:] = a * s + b * c
 
 
-def make_workload(cfg: int | dict, device="cuda", *, B=None, ctx=None, Hq=None, Hkv=None, seed=None,
+def make_workload(cfg: str | dict, device="cuda", *, B=None, ctx=None, Hq=None, Hkv=None, seed=None,
                   mixed=None, mask=None, rope=None, extra_pages: int = 0, perm_seed=None) -> Workload:
     """Build a seeded workload; keyword overrides shrink a config for parity tests.
 
     perm_seed (optional) draws the physical page permutation from its own
     generator, leaving every other draw unchanged."""
-    c = dict(CONFIGS[cfg]) if isinstance(cfg, int) else dict(cfg)
+    c = dict(WORKLOADS[cfg]) if isinstance(cfg, str) else dict(cfg)
     for k_, v_ in dict(B=B, ctx=ctx, Hq=Hq, Hkv=Hkv, seed=seed, mixed=mixed, mask=mask, rope=rope).items():
         if v_ is not None:
             c[k_] = v_

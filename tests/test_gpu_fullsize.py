@@ -23,10 +23,10 @@ def spkv():
 
 
 @pytest.mark.parametrize("cfg,groups", [
-    (1, [(0, 0), (7, 7), (3, 5)]),
-    (2, [(0, 0), (0, 6)]),
-    (3, [(0, 0), (31, 7), (17, 3)]),
-    (4, [(0, 0), (15, 7)]),
+    ("llama3_8b_b8_h32x8_t32768_b4", [(0, 0), (7, 7), (3, 5)]),
+    ("long_b1_h32x8_t131072_b4", [(0, 0), (0, 6)]),
+    ("ragged_rdr_b32_h32x8_t1k-64k_mixed_b_mask25", [(0, 0), (31, 7), (17, 3)]),
+    ("70b_b16_h64x8_t16384_b4_encode", [(0, 0), (15, 7)]),
 ])
 def test_full_size_sampled_parity(spkv, cfg, groups):
     m, synthetic, workload = spkv

@@ -21,6 +21,10 @@ pytestmark = pytest.mark.gpu
 
 OUT_TOL = 2e-3
 FB_TOL = 1e-4
+# workload shapes (compressed_kv_decode_ada_b200.synthetic.WORKLOADS), shrunk per test
+TINY = "tiny_b1_h1_t4096_b4"
+LLAMA = "llama3_8b_b8_h32x8_t32768_b4"
+RAGGED = "ragged_rdr_b32_h32x8_t1k-64k_mixed_b_mask25"
 
 
 @pytest.fixture(scope="module")
@@ -77,12 +81,12 @@ def _check_codes(wl, cache, groups):
 
 
 def test_encode_codes_bit_exact_tiny(spkv):
-    wl, cache = _build(spkv, 0)
+    wl, cache = _build(spkv, TINY)
     _check_codes(wl, cache, helpers.all_groups(wl))
 
 
 def test_encode_codes_bit_exact_mixed_tiers(spkv):
-    wl, cache = _build(spkv, 3, B=6, ctx=("loguniform", 17, 1500))
+    wl, cache = _build(spkv, RAGGED, B=6, ctx=("loguniform", 17, 1500))
     assert set(np.unique(wl.page_bits)) == {3, 4, 6, 8}
     _check_codes(wl, cache, helpers.all_groups(wl))
 
@@ -90,7 +94,7 @@ def test_encode_codes_bit_exact_mixed_tiers(spkv):
 def test_encode_append_in_steps_matches_one_shot(spkv):
     """Appending a sequence one token (then 5 tokens) at a time gives the same bytes."""
     m, synthetic, workload = spkv
-    wl, cache = _build(spkv, 3, B=2, ctx=[37, 50], mask=False)
+    wl, cache = _build(spkv, RAGGED, B=2, ctx=[37, 50], mask=False)
     ref = cache.arena.clone()
     cache2 = m.SpkvCache(wl.num_pages, wl.Hkv, wl.page_bits, wl.rad_lo, wl.rad_step)
     for b in range(wl.B):
@@ -111,7 +115,7 @@ def test_encode_append_in_steps_matches_one_shot(spkv):
 # ------------------------------------------------------------------ decode
 
 def test_decode_parity_tiny(spkv):
-    wl, cache = _build(spkv, 0)
+    wl, cache = _build(spkv, TINY)
     out = _decode(spkv, wl, cache).cpu().numpy()
     err = helpers.max_abs_diff_groups(out, wl, helpers.all_groups(wl), helpers.oracle_seq)
     assert err <= OUT_TOL, err
@@ -123,14 +127,14 @@ def test_decode_parity_tiny(spkv):
     dict(B=2, ctx=[777, 3001], Hq=4, Hkv=2),           # G = 2
 ])
 def test_decode_parity_small_shapes(spkv, kw):
-    wl, cache = _build(spkv, 1, **kw)
+    wl, cache = _build(spkv, LLAMA, **kw)
     out = _decode(spkv, wl, cache).cpu().numpy()
     err = helpers.max_abs_diff_groups(out, wl, helpers.all_groups(wl), helpers.oracle_seq)
     assert err <= OUT_TOL, err
 
 
 def test_decode_parity_mixed_tiers_and_mask(spkv):
-    wl, cache = _build(spkv, 3, B=5, ctx=("loguniform", 20, 5000))
+    wl, cache = _build(spkv, RAGGED, B=5, ctx=("loguniform", 20, 5000))
     out = _decode(spkv, wl, cache).cpu().numpy()
     err = helpers.max_abs_diff_groups(out, wl, helpers.all_groups(wl), helpers.oracle_seq)
     assert err <= OUT_TOL, err
@@ -139,7 +143,7 @@ def test_decode_parity_mixed_tiers_and_mask(spkv):
 def test_debug_logits_parity(spkv):
     """|d f_b| <= 1e-4: logits within 1e-4 ||q|| r~ / sqrt(d) of the oracle's."""
     m = spkv[0]
-    wl, cache = _build(spkv, 3, B=3, ctx=[300, 1200, 64], Hq=8, Hkv=2)
+    wl, cache = _build(spkv, RAGGED, B=3, ctx=[300, 1200, 64], Hq=8, Hkv=2)
     lg = m.debug_logits(cache, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx).cpu().numpy()
     for b, h in helpers.all_groups(wl):
         n = int(wl.ctx[b])
@@ -162,7 +166,7 @@ def _reorder_tol(wl):
 
 
 def test_split_count_invariance(spkv):
-    wl, cache = _build(spkv, 3, B=4, ctx=("loguniform", 100, 4000))
+    wl, cache = _build(spkv, RAGGED, B=4, ctx=("loguniform", 100, 4000))
     ref = _decode(spkv, wl, cache, num_splits=1)
     for s in (2, 7, 33, 0):
         out = _decode(spkv, wl, cache, num_splits=s)
@@ -170,15 +174,15 @@ def test_split_count_invariance(spkv):
 
 
 def test_block_table_permutation_invariance(spkv):
-    wl1, c1 = _build(spkv, 3, B=3, ctx=[500, 1700, 33], extra_pages=7, perm_seed=11)
-    wl2, c2 = _build(spkv, 3, B=3, ctx=[500, 1700, 33], extra_pages=7, perm_seed=12)
+    wl1, c1 = _build(spkv, RAGGED, B=3, ctx=[500, 1700, 33], extra_pages=7, perm_seed=11)
+    wl2, c2 = _build(spkv, RAGGED, B=3, ctx=[500, 1700, 33], extra_pages=7, perm_seed=12)
     assert not np.array_equal(wl1.block_table_np, wl2.block_table_np)
     o1, o2 = _decode(spkv, wl1, c1), _decode(spkv, wl2, c2)
     assert torch.max(torch.abs(o1 - o2)).item() <= _reorder_tol(wl1)
 
 
 def test_bf16_output_matches_fp32(spkv):
-    wl, cache = _build(spkv, 1, B=2, ctx=[2000, 900])
+    wl, cache = _build(spkv, LLAMA, B=2, ctx=[2000, 900])
     o32 = _decode(spkv, wl, cache)
     o16 = _decode(spkv, wl, cache, out_dtype=torch.bfloat16)
     # round-to-nearest bf16: at most half a unit in the last place (2^-8 relative)
@@ -189,7 +193,7 @@ def test_bf16_output_matches_fp32(spkv):
 
 def test_empty_and_fully_evicted_sequences_give_zero(spkv):
     m = spkv[0]
-    wl, cache = _build(spkv, 1, B=3, ctx=[0, 40, 300], Hq=4, Hkv=1)
+    wl, cache = _build(spkv, LLAMA, B=3, ctx=[0, 40, 300], Hq=4, Hkv=1)
     # evict every slot of sequence 1
     km = cache.keep_mask if cache.keep_mask is not None else torch.full(
         (wl.num_pages, wl.Hkv), -1, dtype=torch.int16, device="cuda")
@@ -206,7 +210,7 @@ def test_empty_and_fully_evicted_sequences_give_zero(spkv):
 
 def test_context_beyond_max_ctx_sets_flag_and_zero(spkv):
     m = spkv[0]
-    wl, cache = _build(spkv, 1, B=2, ctx=[64, 64], Hq=4, Hkv=1)
+    wl, cache = _build(spkv, LLAMA, B=2, ctx=[64, 64], Hq=4, Hkv=1)
     ctx = torch.tensor([64, 64], dtype=torch.int32, device="cuda")
     out = m.decode_attention(cache, wl.q, wl.block_table, ctx, 32)  # max_ctx too small
     torch.cuda.synchronize()
@@ -216,7 +220,7 @@ def test_context_beyond_max_ctx_sets_flag_and_zero(spkv):
 
 def test_bad_page_id_and_bad_header_are_flagged_not_fatal(spkv):
     m = spkv[0]
-    wl, cache = _build(spkv, 1, B=2, ctx=[100, 100], Hq=4, Hkv=1)
+    wl, cache = _build(spkv, LLAMA, B=2, ctx=[100, 100], Hq=4, Hkv=1)
     bt = wl.block_table.clone()
     bt[0, 2] = wl.num_pages + 5
     cache.clear_errors()
@@ -241,7 +245,7 @@ def test_bad_page_id_and_bad_header_are_flagged_not_fatal(spkv):
 
 def test_dense_decode_parity(spkv):
     m, synthetic, workload = spkv
-    wl = synthetic.make_workload(3, device="cuda", B=4, ctx=("loguniform", 30, 3000))
+    wl = synthetic.make_workload(RAGGED, device="cuda", B=4, ctx=("loguniform", 30, 3000))
     kp, vp = workload.dense_pages(wl)
     km = torch.from_numpy(wl.keep_mask.view(np.int16)).cuda()
     out = m.dense_decode(kp, vp, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx, keep_mask=km).cpu().numpy()
@@ -251,7 +255,7 @@ def test_dense_decode_parity(spkv):
 
 def test_decompress_then_dot_parity(spkv):
     m = spkv[0]
-    wl, cache = _build(spkv, 3, B=3, ctx=("loguniform", 30, 2500))
+    wl, cache = _build(spkv, RAGGED, B=3, ctx=("loguniform", 30, 2500))
     ks = torch.zeros_like(cache.v_pages)
     out = m.decompress_then_dot(cache, ks, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx).cpu().numpy()
     err = helpers.max_abs_diff_groups(out, wl, helpers.all_groups(wl), helpers.oracle_seq_decompress)
