@@ -27,7 +27,9 @@ EXPORTS = (
     "spkv_dense_decode",
     "spkv_decompress_then_dot",
     "spkv_debug_logits",
+    "spkv_decode_attention_static_ws",
 )
+STATIC_WS_BYTES = 16 * 1024 * 1024  # SPKV_STATIC_WS_BYTES
 
 
 class SpkvError(RuntimeError):
@@ -83,6 +85,9 @@ def _load():
     L.spkv_decompress_then_dot.restype = ctypes.c_int
     L.spkv_decompress_then_dot.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _P, _I, _I, _P, _I, _P, _I, _P, _I,
                                            _P, ctypes.c_size_t, _I, _P]
+    L.spkv_decode_attention_static_ws.restype = ctypes.c_int
+    L.spkv_decode_attention_static_ws.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _I, _I, _P, _I, _P, _I, _P, _I,
+                                                  _I, _P]
     L.spkv_debug_logits.restype = ctypes.c_int
     L.spkv_debug_logits.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _I, _I, _P, _I, _P, _I, _P, _P]
     return L

@@ -109,6 +109,25 @@ def decode_attention(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tenso
     return out
 
 
+def decode_attention_static_ws(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tensor,
+                               ctx_lens: torch.Tensor, max_ctx: int, out=None, out_dtype=torch.float32,
+                               num_splits: int = 0, stream=None) -> torch.Tensor:
+    """spkv_decode_attention_static_ws: ADA decode for callers that cannot allocate
+    device memory while decoding -- the workspace is the library's own fixed
+    device array (SPKV_STATIC_WS_BYTES), shared by every call on the device, so
+    calls must not overlap on the GPU.  `out` may be preallocated to make the
+    call allocation-free on the Python side too."""
+    _batch_checks(q, block_table, ctx_lens)
+    B, Hq, _ = q.shape
+    out = _out_buffer(out, B, Hq, out_dtype, q.device)
+    c = cache.c_struct()
+    check(lib.spkv_decode_attention_static_ws(ctypes.byref(c), _ptr(q), B, Hq, _ptr(block_table),
+                                              block_table.shape[1], _ptr(ctx_lens), int(max_ctx), _ptr(out),
+                                              int(out.dtype == torch.bfloat16), int(num_splits), _stream(stream)),
+          "spkv_decode_attention_static_ws")
+    return out
+
+
 def dense_decode(k_pages: torch.Tensor, v_pages: torch.Tensor, q: torch.Tensor, block_table: torch.Tensor,
                  ctx_lens: torch.Tensor, max_ctx: int, keep_mask=None, err=None, out=None,
                  out_dtype=torch.float32, ws=None, num_splits: int = 0, stream=None) -> torch.Tensor:

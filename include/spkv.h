@@ -183,6 +183,36 @@ SPKV_API spkv_status spkv_decompress_then_dot(const spkv_cache *cache, uint16_t 
                                      const int32_t *ctx_lens, int32_t max_ctx, void *out, int32_t out_is_bf16,
                                      void *ws, size_t ws_bytes, int32_t num_splits, void *stream);
 
+/* Size of the library-owned workspace used by spkv_decode_attention_static_ws
+ * (bytes, per device). */
+#define SPKV_STATIC_WS_BYTES (16u * 1024u * 1024u)
+
+/* ADA decode attention for callers that cannot allocate device memory while
+ * they decode (a fixed memory budget checked at start-up, an allocator that
+ * is not reachable from the decoding thread, a host program that must not
+ * call the CUDA allocator after initialisation).  The summary pages have no
+ * counterpart of this entry point: it is spkv_decode_attention with its
+ * split-partials workspace taken from an array of SPKV_STATIC_WS_BYTES that
+ * the library holds in device memory on every device that loads it, until
+ * the process exits; it allocates nothing itself.
+ *   Arguments and results: as spkv_decode_attention, without ws / ws_bytes.
+ *   Limit: returns SPKV_ERR_WORKSPACE when spkv_decode_workspace_bytes(B,
+ *   num_q_heads, H_kv, max_ctx, num_splits) exceeds SPKV_STATIC_WS_BYTES
+ *   (e.g. B = 8, 32 query / 8 kv heads and the default split count need
+ *   about 4.6 MB).
+ *   Set-up: the first call on a device, with that device current, looks up
+ *   the array's device address (cudaGetSymbolAddress) and caches it; make
+ *   that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array, and each call
+ *   overwrites what the previous one left there (nothing in it needs to start
+ *   at zero).  Calls whose kernels overlap on the GPU (different streams, no
+ *   ordering between them) race on the array and give wrong results. */
+SPKV_API spkv_status spkv_decode_attention_static_ws(const spkv_cache *cache, const uint16_t *q, int32_t B,
+                                                     int32_t num_q_heads, const int32_t *block_table,
+                                                     int32_t max_pages, const int32_t *ctx_lens,
+                                                     int32_t max_ctx, void *out, int32_t out_is_bf16,
+                                                     int32_t num_splits, void *stream);
+
 /* Test hook: the ADA logits themselves (natural-log units, before softmax),
  * logits[b, hq, t] for t < ctx_lens[b]; evicted slots get -inf; entries at or
  * beyond ctx_lens[b] are not written.  logits: [B, Hq, max_ctx] fp32, device. */
