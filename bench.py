@@ -62,6 +62,34 @@ def _cores():
         return os.cpu_count() or 1
 
 
+# ------------------------------------------------------- rank helpers
+def rank_workload(workload: str, rank: int) -> dict:
+    """The batch a rank decodes: the named workload shape with its own seed
+    (ranks decode independent sequences; there is no exchange between them)."""
+    from compressed_kv_decode_ada_b200 import synthetic
+
+    cfg = dict(synthetic.WORKLOADS[workload])
+    cfg["seed"] = int(cfg["seed"]) + 1000 * rank
+    return cfg
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings (all ranks take this collective)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_per_step_max: float) -> float:
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return units_per_rank * world / (ms_per_step_max * 1e-3)
+
+
 # --------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
@@ -128,8 +156,7 @@ def run_spkv(args, rank, world, local):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    cfg = dict(synthetic.WORKLOADS[args.workload])
-    cfg["seed"] = int(cfg["seed"]) + 1000 * rank  # each rank: its own independent batch
+    cfg = rank_workload(args.workload, rank)
     if args.B:
         cfg["B"] = args.B  # smaller batch, for profiler captures only
     wl = synthetic.make_workload(cfg, device=dev)
@@ -181,10 +208,7 @@ def run_spkv(args, rank, world, local):
     total_ms = t_start.elapsed_time(t_end)
     dec_ms = sum(a.elapsed_time(b) for a, b in ev_dec) / args.steps
     ms_step = total_ms / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step, dec_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, dec_ms = float(t[0]), float(t[1])
+    ms_step, dec_ms = max_over_ranks([ms_step, dec_ms], device=dev)
     clocks = clk.summary()
 
     # ---------------- end to end through the public API with host buffers
@@ -206,10 +230,7 @@ def run_spkv(args, rank, world, local):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    (e2e_ms,) = max_over_ranks([e2e_ms], device=dev)
     if cache.error_flags():
         raise RuntimeError(f"device error flags {cache.error_flags():#x}")
 
@@ -228,7 +249,7 @@ def run_spkv(args, rank, world, local):
         d2h = out_h.numel() * out_h.element_size()
         result = {
             "metric": "ADA decode KV tokens/s on 1 B200; achieved HBM GB/s as % of peak",
-            "value": tokens * world / (ms_step * 1e-3),
+            "value": whole_job_rate(tokens, world, ms_step),
             "unit": "KV tokens/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -250,7 +271,7 @@ def run_spkv(args, rank, world, local):
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS,
                          "traffic": traffic, "decode_ms": dec_ms},
-            "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": whole_job_rate(tokens, world, e2e_ms), "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": 3 * args.steps,
             "clocks": clocks,
