@@ -348,7 +348,7 @@ def _committed_traffic(workload):
     ent = d.get(workload)
     if not ent or ent.get("decode_cu_sha256_16") != sha:
         return None
-    return ent.get("dram_bytes_per_step")
+    return ent.get("dram_bytes_per_launch")
 
 
 # ------------------------------------------------------------ CPU oracle arm
