@@ -7,8 +7,8 @@
 namespace spkv {
 
 // Tensor map of a bf16 value-page array [num_pages, H_kv, 16, 128] seen as a
-// 2-D tensor of rows x 128 columns, with boxes of 16 rows x 64 columns
-// (128 bytes wide) and the 128-byte shared-memory swizzle.  The encoder is
+// 3-D tensor (64 columns of a half row, token row, half) whose box {64, 16, 2}
+// is one whole page, with the 128-byte shared-memory swizzle.  The encoder is
 // obtained from the driver through the runtime (no link against libcuda).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -25,11 +25,14 @@ bool make_value_tensor_map(CUtensorMap *map, const void *v_pages, uint64_t rows)
     fn = reinterpret_cast<EncodeTiledFn>(f);
   }
   if (rows == 0 || rows > 0xffffffffull) return false;
-  const cuuint64_t dims[2] = {128, rows};
-  const cuuint64_t strides[1] = {256};
-  const cuuint32_t box[2] = {64, 16};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(v_pages), dims, strides, box, estr,
+  // (dim 64 within a half row, token row, half): one box {64, 16, 2} is a
+  // whole 16 x 128 page, landing as [half][token][64] so that each 128-byte
+  // line of the 128-byte swizzle is (half, token)
+  const cuuint64_t dims[3] = {64, rows, 2};
+  const cuuint64_t strides[2] = {256, 128};
+  const cuuint32_t box[3] = {64, 16, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(v_pages), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -47,6 +47,7 @@ bool make_value_tensor_map(CUtensorMap *map, const void *v_pages, uint64_t rows)
 namespace {
 
 constexpr int kNCWMax = 6;                   // largest consumer-warp count of any path
+constexpr int kIssue = 8;                    // units the producer warp issues per step
 constexpr float kRescaleSlack = 8.0f;        // log2 units a running max may lag the true max
 #define kNegInf (-__int_as_float(0x7f800000))
 
@@ -109,7 +110,7 @@ __device__ __forceinline__ float warp_max(float x) {
 }
 
 // ----------------------------------------------------------------- layout
-template <bool ADA, int G>
+template <bool ADA, int G, bool NW = false>
 struct Layout {
   // 5 consumer warps take PAIRS of units (ADA: the two pages of a pair that
   // share a tier b <= 4 share every query load).  The producer warp streams
@@ -118,15 +119,22 @@ struct Layout {
   // fetches the value pages of its pair itself, into two private slots, when
   // it starts the pair, so the V loads overlap the logit computation and a
   // ring stage is released as soon as the logits are done.
-  static constexpr int NCW = 5;
+  static constexpr int NCW = (ADA && G <= 4) ? 5 : 4;
   static constexpr int THREADS = (NCW + 1) * 32;               // + producer warp
-  static constexpr int NST = ADA ? (G == 8 ? 16 : 20) : (G == 8 ? 13 : 14);
+  // NW ("narrow", ADA only): every page has b <= 4, so a stage holds at most
+  // a 1040-byte record and the ring has twice the stages in the same bytes.
+  static constexpr int NST = ADA ? (NW ? (G == 8 ? 32 : 40) : (G == 8 ? 16 : 20)) : 16;
+  static_assert(NST >= kIssue, "one producer step must touch distinct stages");
+  // Pair i uses stages 2i, 2i + 1 (mod NST) and belongs to warp i % NCW, so
+  // with NST / 2 a multiple of NCW every use of a stage is by one warp, in
+  // order: its parity waits always target the current or the next phase.
+  static_assert((NST / 2) % NCW == 0, "a stage must belong to one consumer warp");
   // Value pages land through two 2-D TMA boxes (16 rows x 64 bf16, 128-byte
   // swizzle): box j holds dims 64 j .. 64 j + 63, row t's 16-byte chunk c
   // sits at chunk c ^ (t & 7), so the transposing ldmatrix reads of 8
   // consecutive rows hit 8 distinct bank groups.  1024-byte aligned.
   static constexpr int VSLOT = 4096;
-  static constexpr int XSTAGE = ADA ? 2064 : 4096;             // code record | dense K page
+  static constexpr int XSTAGE = ADA ? (NW ? 1040 : 2064) : 4096;  // code record | dense K page
   static constexpr int QT_HALF = ADA ? (64 * G + 4) : 8 * (8 * G + 4);  // floats, +16 B skew
   static constexpr int QT_TIER = 2 * QT_HALF;
   static constexpr int QT_FLOATS = (ADA ? kTiers : 1) * QT_TIER;
@@ -175,6 +183,7 @@ struct SplitParams {
   const int32_t *ctx_lens;
   int max_ctx;
   float *ws;
+  uint32_t *row_done;  // per kv row: consumer-warp partials written (zeroed before the launch)
 };
 
 // Stage metadata written by the producer, read by the consumer.
@@ -562,10 +571,10 @@ __device__ __forceinline__ void dense_page_logits(const uint8_t *kpage, const fl
 // the path); m is in log2 units.
 constexpr int kPartial = 132;
 
-template <bool ADA, int G>
-__global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
+template <bool ADA, int G, bool NW>
+__global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
     split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap vmap) {
-  using Ly = Layout<ADA, G>;
+  using Ly = Layout<ADA, G, NW>;
   constexpr int NCW = Ly::NCW, NST = Ly::NST;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -580,7 +589,7 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
   float *sc = reinterpret_cast<float *>(smem + Ly::off_sc);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + Ly::off_bar);
   uint64_t *empty = full + NST;
-  uint64_t *vbar_all = empty + NST;  // 2 per consumer warp
+  uint64_t *vbar_all = empty + NST;  // 1 per consumer warp
   StageMeta *meta = reinterpret_cast<StageMeta *>(smem + Ly::off_meta);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Ly::off_misc);
   int32_t *scratch = reinterpret_cast<int32_t *>(smem + Ly::off_misc + 16);
@@ -589,6 +598,9 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int C = gridDim.x, c = blockIdx.x;
 
+  // the merge grid may be launched now: its blocks only take SMs that this
+  // grid's CTAs leave, and each waits for the rows it merges
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   build_prefix(p.ctx_lens, p.B, p.Hkv, p.max_ctx, p.max_pages, p.err, P, scratch, tid, Ly::THREADS);
   const int64_t W = P[p.B];
   const int64_t u0 = split_begin(W, C, c), u1 = split_begin(W, C, c + 1);
@@ -599,7 +611,7 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int v = 0; v < 2 * NCW; ++v) mbar_init(&vbar_all[v], 1);
+    for (int v = 0; v < NCW; ++v) mbar_init(&vbar_all[v], 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -680,12 +692,13 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
       const uint32_t live = bc.keep & ((1u << ac.ntok) - 1u);
       an = phaseA(kb + 32);
       const int cnt = min(32, n_units - kb);
-      for (int i = 0; i < cnt; ++i) {
-        if (i == 16) bn = phaseB(an);
-        const int k = kb + i;
-        const int s = k % NST, r = k / NST;
-        if (r > 0) mbar_wait_bounded(&empty[s], (uint32_t)(r - 1) & 1u, abort_flag, p.err, 64);
-        if (lane == i) {
+      // lanes [i0, i0 + kIssue) wait for their own stages and issue together
+      for (int i0 = 0; i0 < cnt; i0 += kIssue) {
+        if (i0 == 16) bn = phaseB(an);
+        const int k = kb + lane, s = k % NST, r = k / NST;
+        const bool mine = lane >= i0 && lane < i0 + kIssue && lane < cnt;
+        if (mine) {
+          if (r > 0) mbar_wait_sleepy(&empty[s], (uint32_t)(r - 1) & 1u, abort_flag, p.err);
           StageMeta m;
           m.valid = valid && !*abort_flag;
           m.bits = bc.bits;
@@ -706,9 +719,9 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
             mbar_arrive(&full[s]);
           }
         }
-        k_last = k;
         __syncwarp();
       }
+      k_last = kb + cnt - 1;
       if (cnt <= 16) bn = phaseB(an);
     }
     // On an abort, copies may still be in flight into our stages: wait for
@@ -731,9 +744,9 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
   float *pbuf = pbuf_all + wid * (G * 2 * kPage);
   const int grp = lane >> 2, tig = lane & 3;
   uint8_t *const vslot[2] = {vslot_all + (2 * wid) * Ly::VSLOT, vslot_all + (2 * wid + 1) * Ly::VSLOT};
-  uint64_t *const vbar = vbar_all + 2 * wid;
-  uint32_t vphase[2] = {0u, 0u};
-  int vpending[2] = {-1, -1};  // phase of a value load a failed wait left in flight
+  uint64_t *const vbar = vbar_all + wid;  // the value pages of this warp's pair
+  uint32_t vphase = 0u;
+  int vpending = -1;  // phase of a value load a failed wait left in flight
   int64_t u = u0;
   while (u < u1) {
     const int b = find_seq(P, p.B, u);
@@ -767,7 +780,10 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
 
     float m[G], lsum[G];
     // P.V accumulators in m16n8k16 fragment layout (D^T = V^T P^T):
-    // d[mb][0..1] = dim 16 mb + grp, heads 2 tig, 2 tig + 1; d[mb][2..3] = dim + 8
+    // d[mb][0..1] = dim 16 mb + grp, columns 2 tig, 2 tig + 1; d[mb][2..3] = dim + 8.
+    // Column c is head c (G = 8: P hi and lo in two MMAs), or for G <= 4 the
+    // hi part of head c (c < G) and the lo part of head c - G (G <= c < 2G).
+    constexpr bool kPackPV = G <= 4;
     float d[8][4];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -791,8 +807,12 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
         switch (mt.bits) {
           case 3: ada_page_f<3, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
           case 4: ada_page_f<4, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
-          case 6: ada_page_f<6, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
-          default: ada_page_f<8, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
+          default:
+            if constexpr (!NW) {  // (the producer admits no wider page into a narrow ring)
+              if (mt.bits == 6) ada_page_f<6, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f);
+              else ada_page_f<8, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f);
+            }
+            break;
         }
         const float rad = fast_exp2(fmaf((float)xst[256 * mt.bits + (lane & 15)], Dh, Lh));
 #pragma unroll
@@ -820,9 +840,12 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
       float alpha[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float mx = warp_max(fmaxf(x[0][g], x[1][g]));
+        const float xm = fmaxf(x[0][g], x[1][g]);
         alpha[g] = 1.f;
-        if (mx > m[g] + kRescaleSlack) {  // warp-uniform
+        // the warp max exceeds m + slack iff some lane's does (one vote on
+        // the common path; the max itself only when m moves)
+        if (__any_sync(0xffffffffu, xm > m[g] + kRescaleSlack)) {
+          const float mx = warp_max(xm);
           alpha[g] = m[g] == kNegInf ? 0.f : fast_exp2(m[g] - mx);
           m[g] = mx;
           moved = true;
@@ -835,12 +858,12 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
           pbuf[g * 2 * kPage + kPage + lane] = pb;
         }
       }
-      if (moved) {  // rescale the fragments of heads 2 tig, 2 tig + 1
+      if (moved) {  // rescale the fragments of columns 2 tig, 2 tig + 1
         float a0 = 1.f, a1 = 1.f;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          if (2 * tig == g) a0 = alpha[g];
-          if (2 * tig + 1 == g) a1 = alpha[g];
+          if (2 * tig == g || (kPackPV && 2 * tig == g + G)) a0 = alpha[g];
+          if (2 * tig + 1 == g || (kPackPV && 2 * tig + 1 == g + G)) a1 = alpha[g];
         }
 #pragma unroll
         for (int mb = 0; mb < 8; ++mb) {
@@ -864,14 +887,20 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
           fence_proxy_async_smem();
           __syncwarp();
         }
-        // B = P^T (16 slots x heads) as bf16 hi + lo
+        // B = P^T (16 slots x heads) as bf16 hi + lo: for G <= 4 the hi parts
+        // are columns 0..G-1 and the lo parts columns G..2G-1 of one tile
         uint32_t bh0 = 0u, bh1 = 0u, bl0 = 0u, bl1 = 0u;
-        if (grp < G) {
-          const float *pr = pbuf + grp * 2 * kPage + q * kPage;
+        const int hg = (kPackPV && grp >= G) ? grp - G : grp;
+        if (hg < G) {
+          const float *pr = pbuf + hg * 2 * kPage + q * kPage;
           const float2 pa = *reinterpret_cast<const float2 *>(pr + 2 * tig);
           const float2 pb = *reinterpret_cast<const float2 *>(pr + 2 * tig + 8);
           split_bf16x2(pa.x, pa.y, bh0, bl0);
           split_bf16x2(pb.x, pb.y, bh1, bl1);
+          if (kPackPV && grp >= G) {
+            bh0 = bl0;
+            bh1 = bl1;
+          }
         }
         const int vt = (lane & 7) + 8 * (lane >> 4);  // value row (slot) this lane addresses
         const uint32_t vrow = smem_u32(vs[q]) + (uint32_t)(vt * 128);
@@ -882,7 +911,7 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
           const uint32_t j = 2u * (uint32_t)(mb & 3) + jsel;  // 16-byte chunk within the box row
           ldsm_x4_trans(a, vrow + (uint32_t)(mb >> 2) * 2048u + ((j ^ t7) << 4));
           mma_bf16_16816(d[mb], a, bh0, bh1);
-          mma_bf16_16816(d[mb], a, bl0, bl1);
+          if (!kPackPV) mma_bf16_16816(d[mb], a, bl0, bl1);
         }
       }
     };
@@ -891,6 +920,9 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
     const int ks = (int)(u - u0), ke = (int)(seg_end - u0);
     int i = ks >> 1;
     i += ((wid - i) % NCW + NCW) % NCW;
+    // ready[q]: unit q of this warp's next pair was seen complete one pair
+    // early (a non-blocking test whose latency hides behind the pair's work)
+    bool ready[2] = {false, false};
     for (; 2 * i < ke; i += NCW) {
       const int ka = 2 * i < ks ? ks : 2 * i;
       const int kz = 2 * i + 2 > ke ? ke : 2 * i + 2;  // units [ka, kz) of pair i in this segment
@@ -905,23 +937,25 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
         mt[q] = StageMeta{};
         if (q < n) {
           const int k = ka + q, s = k % NST;
-          const bool ok = mbar_wait_bounded(&full[s], (uint32_t)(k / NST) & 1u, abort_flag, p.err);
+          const bool ok = ready[q] || mbar_wait_bounded(&full[s], (uint32_t)(k / NST) & 1u, abort_flag, p.err);
           mt[q] = meta[s];
           use[q] = ok && mt[q].valid && mt[q].live;
           xst[q] = xst_all + s * Ly::XSTAGE;
         }
       }
-      // the pair's value pages, into this warp's slots (overlaps the logits)
-      if (lane == 0) {
+      {  // the stages' previous phases were this warp's own: the test is exact
+        const int kn = 2 * (i + NCW);
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          if (use[q]) {
-            uint64_t *vb = &vbar[q];
-            mbar_arrive_expect_tx(vb, 4096u);
-            tma_load_2d(vslot[q], &vmap, 0, mt[q].vrow, vb);
-            tma_load_2d(vslot[q] + 2048, &vmap, 64, mt[q].vrow, vb);
-          }
-        }
+        for (int q = 0; q < 2; ++q)
+          ready[q] = kn + q < ke && mbar_test_wait(&full[(kn + q) % NST], (uint32_t)((kn + q) / NST) & 1u);
+      }
+      // the pair's value pages, into this warp's slots (overlaps the logits)
+      const bool vload = use[0] || use[1];
+      if (lane == 0 && vload) {
+        mbar_arrive_expect_tx(vbar, 4096u * ((use[0] ? 1u : 0u) + (use[1] ? 1u : 0u)));
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          if (use[q]) tma_load_3d(vslot[q], &vmap, 0, mt[q].vrow, 0, vbar);
       }
       float l2[2][G];
       bool paired = false;
@@ -959,12 +993,9 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
         mbar_arrive(&empty[ka % NST]);
         if (n == 2) mbar_arrive(&empty[(ka + 1) % NST]);
       }
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        if (use[q]) {
-          if (!mbar_wait_bounded(&vbar[q], vphase[q], abort_flag, p.err)) vpending[q] = (int)vphase[q];
-          vphase[q] ^= 1u;
-        }
+      if (vload) {
+        if (!mbar_wait_bounded(vbar, vphase, abort_flag, p.err)) vpending = (int)vphase;
+        vphase ^= 1u;
       }
       softmax_pv(use, mt, l2, vslot);
       __syncwarp();
@@ -975,6 +1006,17 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
     for (int g = 0; g < G; ++g) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) lsum[g] += __shfl_xor_sync(0xffffffffu, lsum[g], o);
+    }
+    if constexpr (kPackPV) {  // fold the lo columns onto the hi columns
+#pragma unroll
+      for (int mb = 0; mb < 8; ++mb) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (G == 4) d[mb][e] += __shfl_xor_sync(0xffffffffu, d[mb][e], 2);
+          else if constexpr (G == 2) d[mb][e] += __shfl_xor_sync(0xffffffffu, d[mb][e], 1);
+          else if (e == 0 || e == 2) d[mb][e] += d[mb][e + 1];
+        }
+      }
     }
     float *part = p.ws + ((int64_t)(c + bh) * NCW + wid) * G * kPartial;
 #pragma unroll
@@ -993,15 +1035,17 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
         }
       }
     }
+    // publish the partial: every lane's stores, then one count on the row
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) atomicAdd(p.row_done + bh, 1u);
     u = seg_end;
   }
   // After an abort a value load of this warp may still be landing in its
   // slots: wait for it (bounded) before the shared memory is released.
-  if (lane == 0) {
+  if (lane == 0 && vpending >= 0) {
     volatile int dummy = 0;
-#pragma unroll
-    for (int q = 0; q < 2; ++q)
-      if (vpending[q] >= 0) mbar_wait_bounded(&vbar[q], (uint32_t)vpending[q], &dummy, nullptr);
+    mbar_wait_bounded(vbar, (uint32_t)vpending, &dummy, nullptr);
   }
 }
 
@@ -1009,21 +1053,24 @@ __global__ void __launch_bounds__(Layout<ADA, G>::THREADS, 2)
 // One block per (sequence, query head): combine the partials of every
 // (split, consumer warp) that covered the head's kv row.
 //   out = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s   (0 when nothing
-// was retained).  The partials' (m, l) are loaded in parallel into shared
-// memory, then each thread sums its dimension over all partials.
+// was retained).  Launched as a programmatic dependent of the split kernel:
+// a block starts on an SM the split grid has left and waits (bounded) until
+// the row's count of written partials reaches NCW per covering split, so the
+// rows that finish early are merged while the last splits still run.
 template <int G>
-__global__ void __launch_bounds__(128) merge_kernel(const float *ws, int C, int NCW, const int32_t *ctx_lens, int B,
-                                                    int Hkv, int Hq, int max_ctx, int max_pages, void *out,
-                                                    int out_bf16) {
+__global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint32_t *row_done, int C, int NCW,
+                                                    const int32_t *ctx_lens, int B, int Hkv, int Hq, int max_ctx,
+                                                    int max_pages, void *out, int out_bf16, uint32_t *err) {
   constexpr int kChunk = 256;  // partials per pass
   __shared__ int64_t red[2][4];
   __shared__ float wgt[kChunk];
   __shared__ float lsh[kChunk];
   __shared__ int64_t off[kChunk];
-  __shared__ float Msh;
+  __shared__ float mred[4];
+  __shared__ uint32_t nred[4];
   const int hq = blockIdx.x % Hq, b = blockIdx.x / Hq;
   const int h = hq / G, g = hq % G, bh = b * Hkv + h;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   int64_t before = 0, total = 0;
   for (int i = tid; i < B; i += 128) {
     const int np = seq_pages(ctx_lens[i], max_ctx, max_pages, nullptr) * Hkv;
@@ -1035,9 +1082,9 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, int C, int 
     before += __shfl_xor_sync(0xffffffffu, before, o);
     total += __shfl_xor_sync(0xffffffffu, total, o);
   }
-  if ((tid & 31) == 0) {
-    red[0][tid >> 5] = before;
-    red[1][tid >> 5] = total;
+  if (lane == 0) {
+    red[0][wid] = before;
+    red[1][wid] = total;
   }
   __syncthreads();
   before = red[0][0] + red[0][1] + red[0][2] + red[0][3];
@@ -1049,29 +1096,47 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, int C, int 
     const int64_t cf = ((a + 1) * C + W - 1) / W - 1;
     int64_t cl = (e * C + W - 1) / W - 1;
     if (cl > C - 1) cl = C - 1;
+    // splits that hold units of the row (every split in [cf, cl] but empty ones)
+    uint32_t live = 0;
+    for (int64_t cc = cf + tid; cc <= cl; cc += 128)
+      live += split_begin(W, C, (int)cc) < split_begin(W, C, (int)cc + 1) ? 1u : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) live += __shfl_xor_sync(0xffffffffu, live, o);
+    if (lane == 0) nred[wid] = live;
+    __syncthreads();
+    const uint32_t expected = (nred[0] + nred[1] + nred[2] + nred[3]) * (uint32_t)NCW;
+    if (tid == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      uint32_t seen;
+      for (;;) {
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(row_done + bh) : "memory");
+        if (seen >= expected) break;
+        if (globaltimer_ns() - t0 > 1000000000ull) {
+          set_err(err, SPKV_DEVERR_TIMEOUT);
+          break;
+        }
+        __nanosleep(256);
+      }
+    }
+    __syncthreads();
     const int64_t nparts = (cl - cf + 1) * NCW;
     float M = kNegInf;
-    // pass 1: the running max over all partials
-    for (int64_t base = 0; base < nparts; base += kChunk) {
-      for (int i = tid; i < kChunk; i += 128) {
-        float mm = kNegInf;
-        if (base + i < nparts) {
-          const int64_t cc = cf + (base + i) / NCW;
-          const int w = (int)((base + i) % NCW);
-          if (split_begin(W, C, (int)cc) < split_begin(W, C, (int)cc + 1))
-            mm = ws[(((cc + bh) * NCW + w) * G + g) * kPartial];
-        }
-        wgt[i] = mm;
+    // pass 1: the max over all partials
+    for (int64_t base = 0; base < nparts; base += 128) {
+      float mm = kNegInf;
+      if (base + tid < nparts) {
+        const int64_t cc = cf + (base + tid) / NCW;
+        const int w = (int)((base + tid) % NCW);
+        if (split_begin(W, C, (int)cc) < split_begin(W, C, (int)cc + 1))
+          mm = __ldcg(ws + (((cc + bh) * NCW + w) * G + g) * kPartial);
       }
-      __syncthreads();
-      if (tid == 0) {
-        for (int i = 0; i < kChunk && base + i < nparts; ++i) M = fmaxf(M, wgt[i]);
-      }
-      __syncthreads();
+      M = fmaxf(M, mm);
     }
-    if (tid == 0) Msh = M;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) mred[wid] = M;
     __syncthreads();
-    M = Msh;
+    M = fmaxf(fmaxf(mred[0], mred[1]), fmaxf(mred[2], mred[3]));
     if (M != kNegInf) {
       for (int64_t base = 0; base < nparts; base += kChunk) {
         for (int i = tid; i < kChunk; i += 128) {
@@ -1082,10 +1147,10 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, int C, int 
             const int w = (int)((base + i) % NCW);
             if (split_begin(W, C, (int)cc) < split_begin(W, C, (int)cc + 1)) {
               o = (((cc + bh) * NCW + w) * G + g) * kPartial;
-              const float mm = ws[o];
-              if (mm != kNegInf) {
-                wv = fast_exp2(mm - M);
-                lv = ws[o + 1];
+              const float2 ml = __ldcg(reinterpret_cast<const float2 *>(ws + o));
+              if (ml.x != kNegInf) {
+                wv = fast_exp2(ml.x - M);
+                lv = ml.y;
               } else {
                 o = -1;
               }
@@ -1100,7 +1165,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, int C, int 
 #pragma unroll 8
         for (int i = 0; i < n; ++i) {
           if (off[i] >= 0) {
-            num = fmaf(wgt[i], ws[off[i] + 4 + tid], num);
+            num = fmaf(wgt[i], __ldcg(ws + off[i] + 4 + tid), num);
             den = fmaf(wgt[i], lsh[i], den);
           }
         }
@@ -1256,44 +1321,22 @@ __global__ void __launch_bounds__(32) debug_logits_kernel(SplitParams p, float *
 // ------------------------------------------------------------- host side
 // Opt the kernel into the largest dynamic shared memory it can ask for (once
 // per device) and report how many CTAs of `smem` bytes fit on one SM.
-template <bool ADA, int G>
+template <bool ADA, int G, bool NW>
 int blocks_per_sm(size_t smem) {
   static int configured[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
   if (!configured[dev]) {
-    if (cudaFuncSetAttribute(split_kernel<ADA, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)Layout<ADA, G>::bytes(kMaxB)) != cudaSuccess)
+    if (cudaFuncSetAttribute(split_kernel<ADA, G, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Layout<ADA, G, NW>::bytes(kMaxB)) != cudaSuccess)
       return -1;
     configured[dev] = 1;
   }
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<ADA, G>, Layout<ADA, G>::THREADS, smem) !=
-      cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<ADA, G, NW>, Layout<ADA, G, NW>::THREADS,
+                                                    smem) != cudaSuccess)
     return -1;
   return n;
-}
-
-template <bool ADA>
-int blocks_per_sm_for(int G, size_t smem) {
-  switch (G) {
-    case 1: return blocks_per_sm<ADA, 1>(smem);
-    case 2: return blocks_per_sm<ADA, 2>(smem);
-    case 4: return blocks_per_sm<ADA, 4>(smem);
-    case 8: return blocks_per_sm<ADA, 8>(smem);
-  }
-  return -1;
-}
-
-template <bool ADA>
-size_t smem_for(int G, int B) {
-  switch (G) {
-    case 1: return Layout<ADA, 1>::bytes(B);
-    case 2: return Layout<ADA, 2>::bytes(B);
-    case 4: return Layout<ADA, 4>::bytes(B);
-    case 8: return Layout<ADA, 8>::bytes(B);
-  }
-  return 0;
 }
 
 bool g_supported(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
@@ -1317,33 +1360,63 @@ struct DecodeArgs {
   int out_bf16;
 };
 
-template <bool ADA>
-spkv_status launch_split_and_merge(const DecodeArgs &a, cudaStream_t stream) {
-  const size_t smem = smem_for<ADA>(a.G, a.sp.B);
-  if (blocks_per_sm_for<ADA>(a.G, smem) < 1) return SPKV_ERR_CUDA;
-  const int C = a.num_splits;
-  CUtensorMap vmap;
-  if (!make_value_tensor_map(&vmap, a.sp.v_pages, (uint64_t)a.sp.num_pages * a.sp.Hkv * kPage))
-    return a.sp.num_pages == 0 ? SPKV_ERR_INVALID_ARG : SPKV_ERR_CUDA;
-  switch (a.G) {
-    case 1: split_kernel<ADA, 1><<<C, Layout<ADA, 1>::THREADS, smem, stream>>>(a.sp, vmap); break;
-    case 2: split_kernel<ADA, 2><<<C, Layout<ADA, 2>::THREADS, smem, stream>>>(a.sp, vmap); break;
-    case 4: split_kernel<ADA, 4><<<C, Layout<ADA, 4>::THREADS, smem, stream>>>(a.sp, vmap); break;
-    case 8: split_kernel<ADA, 8><<<C, Layout<ADA, 8>::THREADS, smem, stream>>>(a.sp, vmap); break;
-  }
+template <bool ADA, int G, bool NW>
+spkv_status launch_g(const DecodeArgs &a, const CUtensorMap &vmap, cudaStream_t stream) {
+  using Ly = Layout<ADA, G, NW>;
+  const size_t smem = Ly::bytes(a.sp.B);
+  if (blocks_per_sm<ADA, G, NW>(smem) < 1) return SPKV_ERR_CUDA;
+  // the row counters start at zero in every launch
+  if (cudaMemsetAsync(a.sp.row_done, 0, (size_t)a.sp.B * a.sp.Hkv * sizeof(uint32_t), stream) != cudaSuccess)
+    return SPKV_ERR_CUDA;
+  split_kernel<ADA, G, NW><<<a.num_splits, Ly::THREADS, smem, stream>>>(a.sp, vmap);
   if (cudaGetLastError() != cudaSuccess) return SPKV_ERR_CUDA;
-  const int nb = a.sp.B * a.sp.Hq;
-  switch (a.G) {
-    case 1: merge_kernel<1><<<nb, 128, 0, stream>>>(a.sp.ws, C, Layout<ADA, 1>::NCW, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
-    case 2: merge_kernel<2><<<nb, 128, 0, stream>>>(a.sp.ws, C, Layout<ADA, 2>::NCW, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
-    case 4: merge_kernel<4><<<nb, 128, 0, stream>>>(a.sp.ws, C, Layout<ADA, 4>::NCW, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
-    case 8: merge_kernel<8><<<nb, 128, 0, stream>>>(a.sp.ws, C, Layout<ADA, 8>::NCW, a.sp.ctx_lens, a.sp.B, a.sp.Hkv, a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16); break;
-  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.sp.B * a.sp.Hq));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float *ws = a.sp.ws;
+  const uint32_t *done = a.sp.row_done;
+  if (cudaLaunchKernelEx(&cfg, merge_kernel<G>, ws, done, a.num_splits, Ly::NCW, a.sp.ctx_lens, a.sp.B, a.sp.Hkv,
+                         a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16, a.sp.err) != cudaSuccess)
+    return SPKV_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
 }
 
+template <bool ADA, bool NW>
+spkv_status launch_nw(const DecodeArgs &a, const CUtensorMap &vmap, cudaStream_t stream) {
+  switch (a.G) {
+    case 1: return launch_g<ADA, 1, NW>(a, vmap, stream);
+    case 2: return launch_g<ADA, 2, NW>(a, vmap, stream);
+    case 4: return launch_g<ADA, 4, NW>(a, vmap, stream);
+    case 8: return launch_g<ADA, 8, NW>(a, vmap, stream);
+  }
+  return SPKV_ERR_UNSUPPORTED;
+}
+
+// Split + merge launches.  An ADA cache whose pages are all b <= 4 (tier
+// mask within {3, 4}) runs the narrow-stage kernel.
+template <bool ADA>
+spkv_status launch_split_and_merge(const DecodeArgs &a, cudaStream_t stream) {
+  CUtensorMap vmap;
+  if (!make_value_tensor_map(&vmap, a.sp.v_pages, (uint64_t)a.sp.num_pages * a.sp.Hkv * kPage))
+    return a.sp.num_pages == 0 ? SPKV_ERR_INVALID_ARG : SPKV_ERR_CUDA;
+  if constexpr (ADA) {
+    if ((a.sp.tiers & ~0x3u) == 0u) return launch_nw<true, true>(a, vmap, stream);
+  }
+  return launch_nw<ADA, false>(a, vmap, stream);
+}
+
+size_t ws_partials_bytes(int B, int Hq, int Hkv, int C) {
+  return ((size_t)(C + B * Hkv) * kNCWMax * (size_t)(Hq / Hkv) * kPartial * sizeof(float) + 15) / 16 * 16;
+}
 size_t ws_bytes_for(int B, int Hq, int Hkv, int C) {
-  return (size_t)(C + B * Hkv) * kNCWMax * (size_t)(Hq / Hkv) * kPartial * sizeof(float);
+  return ws_partials_bytes(B, Hq, Hkv, C) + ((size_t)B * Hkv * sizeof(uint32_t) + 15) / 16 * 16;
 }
 
 // Shared validation of the batch arguments; fills sp's batch fields.
@@ -1369,6 +1442,7 @@ spkv_status prep_batch(SplitParams &sp, int Hkv, const uint16_t *q, int B, int H
   sp.ctx_lens = ctx_lens;
   sp.max_ctx = max_ctx;
   sp.ws = reinterpret_cast<float *>(ws);
+  sp.row_done = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(ws) + ws_partials_bytes(B, Hq, Hkv, C));
   *G_out = G;
   *C_out = C;
   return SPKV_OK;

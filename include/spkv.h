@@ -133,7 +133,10 @@ SPKV_API spkv_status spkv_encode_keys(const spkv_cache *cache, const uint16_t *k
 SPKV_API int32_t spkv_decode_default_splits(int32_t B, int32_t num_kv_heads, int32_t max_ctx);
 
 /* Workspace bytes needed by spkv_decode_attention / spkv_dense_decode /
- * spkv_decompress_then_dot for these sizes and this split count (0 = default).
+ * spkv_decompress_then_dot for these sizes and this split count (0 = default):
+ * the split partials (rounded up to 16 bytes), then one 4-byte counter per
+ * (sequence, kv head) row (rounded up to 16 bytes) that the call zeroes on
+ * its stream before its kernels run.  The workspace needs no initialisation.
  * Returns 0 for invalid sizes. */
 SPKV_API size_t spkv_decode_workspace_bytes(int32_t B, int32_t num_q_heads, int32_t num_kv_heads,
                                    int32_t max_ctx, int32_t num_splits);

@@ -77,7 +77,12 @@ def test_host_argument_checks(lib):
 
 
 def test_workspace_formula(lib):
-    # (C + B H_kv) segments x 6 consumer warps x G partials of 132 floats
-    assert lib.workspace_bytes(8, 32, 8, 32768, 296) == (296 + 64) * 6 * 4 * 132 * 4
-    assert lib.workspace_bytes(2, 8, 8, 100, 5) == (5 + 16) * 6 * 1 * 132 * 4
+    # (C + B H_kv) segments x 6 consumer-warp slots x G partials of 132 floats
+    # (rounded to 16 bytes), then one 4-byte row counter per kv row (rounded)
+    def want(B, Hq, Hkv, C):
+        part = (C + B * Hkv) * 6 * (Hq // Hkv) * 132 * 4
+        return (part + 15) // 16 * 16 + (B * Hkv * 4 + 15) // 16 * 16
+    assert lib.workspace_bytes(8, 32, 8, 32768, 296) == want(8, 32, 8, 296)
+    assert lib.workspace_bytes(2, 8, 8, 100, 5) == want(2, 8, 8, 5)
+    assert lib.workspace_bytes(3, 8, 1, 100, 5) == want(3, 8, 1, 5)
     assert lib.workspace_bytes(2, 7, 2, 100, 5) == 0  # Hq not a multiple of H_kv
