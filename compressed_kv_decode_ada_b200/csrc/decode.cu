@@ -119,11 +119,11 @@ struct Layout {
   // fetches the value pages of its pair itself, into two private slots, when
   // it starts the pair, so the V loads overlap the logit computation and a
   // ring stage is released as soon as the logits are done.
-  static constexpr int NCW = (ADA && G <= 4) ? 5 : 4;
+  static constexpr int NCW = G <= 4 ? 5 : 4;
   static constexpr int THREADS = (NCW + 1) * 32;               // + producer warp
   // NW ("narrow", ADA only): every page has b <= 4, so a stage holds at most
   // a 1040-byte record and the ring has twice the stages in the same bytes.
-  static constexpr int NST = ADA ? (NW ? (G == 8 ? 32 : 40) : (G == 8 ? 16 : 20)) : 16;
+  static constexpr int NST = ADA ? (NW ? (G == 8 ? 32 : 40) : (G == 8 ? 16 : 20)) : (G <= 4 ? 10 : 16);
   static_assert(NST >= kIssue, "one producer step must touch distinct stages");
   // Pair i uses stages 2i, 2i + 1 (mod NST) and belongs to warp i % NCW, so
   // with NST / 2 a multiple of NCW every use of a stage is by one warp, in
