@@ -75,6 +75,7 @@ def lib():
         L.spkv_oracle_encode.argtypes = [_i, _i, _p, _p, _d, _d, _p, _p, _p, _p]
         L.spkv_oracle_decompress.argtypes = [_i, _i, _p, _p, _p, _d, _d, _p]
         L.spkv_oracle_ada_group.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _d, _d, _p, _p, _p, _p]
+        L.spkv_oracle_ada_group_exact_q.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _d, _d, _p, _p, _p, _p]
         L.spkv_oracle_dense_group.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _p]
         _lib = L
     return _lib
@@ -205,10 +206,12 @@ def decompress(codes: np.ndarray, bits: np.ndarray, rcode: np.ndarray, L: float,
     return out
 
 
-def ada_group(q_bf16, kcodes, kbits, rcode, L, delta, v_bf16, keep=None, r_exact=None, want_logits=False):
+def ada_group(q_bf16, kcodes, kbits, rcode, L, delta, v_bf16, keep=None, r_exact=None, want_logits=False,
+              exact_q=False):
     """ADA attention of G query heads [G, d] against T coded keys of one kv head.
 
     logit = ||q|| r~ f_b(c_q, c_k) / sqrt(d); softmax over retained slots; P.V.
+    exact_q: f = <q/||q||, u~(c_k)> (the unquantised unit query, reading R13).
     Returns out [G, d] (and logits [G, T] with -inf where evicted).
     """
     q = _c(q_bf16, np.uint16)
@@ -222,8 +225,9 @@ def ada_group(q_bf16, kcodes, kbits, rcode, L, delta, v_bf16, keep=None, r_exact
     v = _c(v_bf16, np.uint16)
     out = np.empty((G, d), np.float64)
     lg = np.empty((G, T), np.float64) if want_logits else None
-    lib().spkv_oracle_ada_group(d, G, T, _ptr(q), _ptr(kcodes), _ptr(kbits), _ptr(rcode), _ptr(r_exact),
-                                float(L), float(delta), _ptr(keep), _ptr(v), _ptr(out), _ptr(lg))
+    fn = lib().spkv_oracle_ada_group_exact_q if exact_q else lib().spkv_oracle_ada_group
+    fn(d, G, T, _ptr(q), _ptr(kcodes), _ptr(kbits), _ptr(rcode), _ptr(r_exact), float(L), float(delta), _ptr(keep),
+       _ptr(v), _ptr(out), _ptr(lg))
     return (out, lg) if want_logits else out
 
 

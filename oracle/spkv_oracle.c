@@ -33,6 +33,9 @@
  *       r~ = 2^(L + c_r Delta); L, Delta per kv head; r = 0 gives c_r = 0.
  *   R6  logits are divided by sqrt(d) (standard attention scale).
  *   R7  softmax over retained slots only; an empty set gives a zero output.
+ *   R13 exact-query variant (section 2.1 leaves f_b open; the coded query of
+ *       R3 is the literal reading): f = <q/||q||, u~(c_k)>, the unquantised
+ *       unit query against the decoded key; a zero query gives f = 0.
  * Arithmetic is IEEE fp64 throughout; bf16 inputs are widened exactly and
  * -0 is normalised to +0.
  */
@@ -276,10 +279,10 @@ static void softmax_pv(int d, int T, const double *logit, const uint8_t *keep, c
  *   logits  [G, T]      fp64 logits (natural-log units), -inf where evicted;
  *                       NULL to skip
  * logit(q_g, k_t) = ||q_g|| r~_t f_b(c_q(b_t), c_k(t)) / sqrt(d). */
-void spkv_oracle_ada_group(int d, int G, int T, const uint16_t *q, const int32_t *kcodes,
+static void ada_group_impl(int d, int G, int T, const uint16_t *q, const int32_t *kcodes,
                            const int32_t *kbits, const uint8_t *rcode, const double *r_exact,
                            double L, double Delta, const uint8_t *keep, const uint16_t *v,
-                           double *out, double *logits)
+                           double *out, double *logits, int exact_q)
 {
     double *x = (double *)malloc(sizeof(double) * (size_t)d);
     double *phi = (double *)malloc(sizeof(double) * (size_t)(d - 1));
@@ -298,10 +301,12 @@ void spkv_oracle_ada_group(int d, int G, int T, const uint16_t *q, const int32_t
         }
         double qn = sqrt(qn2);
         spkv_oracle_angles(d, x, phi);
+        if (exact_q) /* R13: the unquantised unit query */
+            for (int j = 0; j < d; ++j) uq[j] = qn > 0.0 ? x[j] / qn : 0.0;
         int qb = -1;
         for (int t = 0; t < T; ++t) {
             int b = kbits[t];
-            if (b != qb) { /* R3: the query is coded at the key's bit width */
+            if (!exact_q && b != qb) { /* R3: the query is coded at the key's bit width */
                 spkv_oracle_angle_codes(d, phi, b, cq);
                 spkv_oracle_unit_from_codes(d, cq, b, uq);
                 qb = b;
@@ -317,6 +322,24 @@ void spkv_oracle_ada_group(int d, int G, int T, const uint16_t *q, const int32_t
             for (int t = 0; t < T; ++t) logits[(size_t)g * T + t] = kp[t] ? lg[t] : -INFINITY;
     }
     free(x); free(phi); free(cq); free(uq); free(uk); free(lg); free(kp);
+}
+
+void spkv_oracle_ada_group(int d, int G, int T, const uint16_t *q, const int32_t *kcodes,
+                           const int32_t *kbits, const uint8_t *rcode, const double *r_exact,
+                           double L, double Delta, const uint8_t *keep, const uint16_t *v,
+                           double *out, double *logits)
+{
+    ada_group_impl(d, G, T, q, kcodes, kbits, rcode, r_exact, L, Delta, keep, v, out, logits, 0);
+}
+
+/* The exact-query variant (R13): as spkv_oracle_ada_group, with
+ * f = <q/||q||, u~(c_k)> in place of the coded query. */
+void spkv_oracle_ada_group_exact_q(int d, int G, int T, const uint16_t *q, const int32_t *kcodes,
+                                   const int32_t *kbits, const uint8_t *rcode, const double *r_exact,
+                                   double L, double Delta, const uint8_t *keep, const uint16_t *v,
+                                   double *out, double *logits)
+{
+    ada_group_impl(d, G, T, q, kcodes, kbits, rcode, r_exact, L, Delta, keep, v, out, logits, 1);
 }
 
 /* Dense attention for G query heads over bf16 keys:

@@ -308,6 +308,78 @@ def test_brute_force_attention_at_high_bit_width():
         assert np.max(np.abs(out[g] - want)) <= 1e-6
 
 
+def _np_unit_from_codes(c, b):
+    """Decoded unit vector, written out independently with numpy: cell
+    midpoints, then cos of each angle times the running product of sines."""
+    c = np.asarray(c, np.float64)
+    d = c.shape[0] + 1
+    phi = (c + 0.5) * math.pi / 2 ** b
+    phi[-1] = (c[-1] + 0.5) * 2 * math.pi / 2 ** b
+    u = np.empty(d)
+    run = 1.0
+    for j in range(d - 1):
+        u[j] = run * math.cos(phi[j])
+        run *= math.sin(phi[j])
+    u[d - 1] = run
+    return u
+
+
+def test_exact_query_logit_is_cosine_with_the_decoded_key():
+    """R13: with the exact query, logit = ||q|| r~ <q/||q||, u~(c_k)> / sqrt d, with
+    the key decoded by an independent numpy routine; mixed widths and a mask."""
+    rng = np.random.default_rng(13)
+    d, T, G = 128, 40, 2
+    q = _rand_bf16(rng, (G, d))
+    keys = _rand_bf16(rng, (T, d), 1.5)
+    v = _rand_bf16(rng, (T, d))
+    bits = rng.choice(BITS, T).astype(np.int32)
+    keep = (rng.random(T) > 0.25).astype(np.uint8)
+    L, delta = -1.0, 7.0 / 255
+    codes, rcode = oracle.encode(keys, bits, L, delta)
+    out, lg = oracle.ada_group(q, codes, bits, rcode, L, delta, v, keep=keep, want_logits=True, exact_q=True)
+    vf = oracle.bf16_to_f64(v)
+    for g in range(G):
+        qf = oracle.bf16_to_f64(q[g])
+        want = np.array([float(qf @ _np_unit_from_codes(codes[t], int(bits[t])))
+                         * 2.0 ** (L + int(rcode[t]) * delta) / math.sqrt(d) for t in range(T)])
+        np.testing.assert_allclose(lg[g][keep == 1], want[keep == 1], rtol=0, atol=1e-12)
+        assert np.all(np.isinf(lg[g][keep == 0]))
+        x = np.where(keep.astype(bool), want, -np.inf)
+        p = np.exp(x - x.max())
+        assert np.max(np.abs(out[g] - (p @ vf) / p.sum())) <= 1e-12
+
+
+def test_exact_query_high_bit_width_matches_dense_attention():
+    """R13 with b = 30 keys and exact radii: only the key angles are quantised,
+    so ADA reaches plain softmax(q K^T / sqrt d) V to about 2^-30."""
+    rng = np.random.default_rng(14)
+    d, T, G = 128, 64, 2
+    q = _rand_bf16(rng, (G, d))
+    keys = _rand_bf16(rng, (T, d))
+    v = _rand_bf16(rng, (T, d))
+    codes, _ = oracle.encode(keys, 30, 0.0, 1.0)
+    kf = oracle.bf16_to_f64(keys)
+    out = oracle.ada_group(q, codes, 30, np.zeros(T, np.uint8), 0.0, 1.0, v,
+                           r_exact=np.linalg.norm(kf, axis=1), exact_q=True)
+    vf = oracle.bf16_to_f64(v)
+    for g in range(G):
+        want = _np_softmax_attention(oracle.bf16_to_f64(q[g]), kf, vf)
+        assert np.max(np.abs(out[g] - want)) <= 1e-7
+
+
+def test_exact_query_zero_query_gives_uniform_attention():
+    """R13: a zero query has f = 0, so every retained slot gets the same weight."""
+    rng = np.random.default_rng(15)
+    d, T = 128, 12
+    q = np.zeros((1, d), np.uint16)
+    keys = _rand_bf16(rng, (T, d))
+    v = _rand_bf16(rng, (T, d))
+    codes, rcode = oracle.encode(keys, 4, 0.0, 4.0 / 255)
+    out, lg = oracle.ada_group(q, codes, 4, rcode, 0.0, 4.0 / 255, v, want_logits=True, exact_q=True)
+    assert np.all(lg == 0.0)
+    assert np.max(np.abs(out[0] - oracle.bf16_to_f64(v).mean(axis=0))) <= 1e-12
+
+
 def test_dense_oracle_brute_force():
     rng = np.random.default_rng(13)
     d, T, G = 128, 50, 4
