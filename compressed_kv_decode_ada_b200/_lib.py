@@ -28,7 +28,10 @@ EXPORTS = (
     "spkv_decompress_then_dot",
     "spkv_debug_logits",
     "spkv_decode_attention_static_ws",
+    "spkv_decode_attention_ex",
+    "spkv_debug_logits_ex",
 )
+DECODE_EXACT_Q = 1  # SPKV_DECODE_EXACT_Q
 STATIC_WS_BYTES = 16 * 1024 * 1024  # SPKV_STATIC_WS_BYTES
 
 
@@ -90,6 +93,12 @@ def _load():
                                                   _I, _P]
     L.spkv_debug_logits.restype = ctypes.c_int
     L.spkv_debug_logits.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _I, _I, _P, _I, _P, _I, _P, _P]
+    L.spkv_decode_attention_ex.restype = ctypes.c_int
+    L.spkv_decode_attention_ex.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _I, _I, _P, _I, _P, _I, _P, _I, _P,
+                                           ctypes.c_size_t, _I, ctypes.c_uint32, _P]
+    L.spkv_debug_logits_ex.restype = ctypes.c_int
+    L.spkv_debug_logits_ex.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _I, _I, _P, _I, _P, _I, _P, ctypes.c_uint32,
+                                       _P]
     return L
 
 

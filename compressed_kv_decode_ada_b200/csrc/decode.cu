@@ -148,8 +148,10 @@ struct Layout {
   static constexpr int off_v = 0;                                 // NCW x 2 value slots
   static constexpr int off_x = off_v + NCW * 2 * VSLOT;           // ring stages
   // float2 single-angle tables: polar at off_lut, azimuth 384 entries later;
-  // off_lut = 64 (mod 128) puts both b = 4 tables (entry 8 on) on 128 bytes
-  static constexpr int off_lut = (off_x + NST * XSTAGE + 127) / 128 * 128 + 64;
+  // off_lut = 192 (mod 256) puts both b = 4 tables (entry 8 on) on 256-byte
+  // boundaries: one 128-byte row each, and an entry's address is the
+  // table's upper bytes with the entry offset as the low byte
+  static constexpr int off_lut = (off_x + NST * XSTAGE + 255) / 256 * 256 + 192;
   static constexpr int LAZ_OFF = 384;  // entries
   static constexpr int lut_bytes = ADA ? (LAZ_OFF + kLutEntries) * 8 : 0;
   static constexpr int off_qt = off_lut + lut_bytes;
@@ -175,6 +177,7 @@ struct SplitParams {
   const uint16_t *keep;
   uint32_t *err;
   uint32_t tiers;  // tiers the query is coded for (bit t: b = {3,4,6,8}[t])
+  uint32_t flags;  // SPKV_DECODE_* bits
   int Hkv, num_pages;
   const uint16_t *q;
   int B, Hq;
@@ -218,7 +221,8 @@ __device__ __forceinline__ void build_luts(float2 *lpol, float2 *laz, int tid, i
 // a = 64 half + 2 pair + e.  Returns ||q||.
 template <int G, int QT_HALF>
 __device__ float ada_qprep_row(const uint16_t *qrow, int g, const float2 *lpol, const float2 *laz,
-                               const double *pol_c2, const double *az_c2, float *qt, int lane, uint32_t tiers) {
+                               const double *pol_c2, const double *az_c2, float *qt, int lane, uint32_t tiers,
+                               bool exact) {
   const uint2 raw = *reinterpret_cast<const uint2 *>(qrow + 4 * lane);
   double x[4], S[4];
   lane_suffix_sums(raw, lane, x, S);
@@ -227,6 +231,16 @@ __device__ float ada_qprep_row(const uint16_t *qrow, int g, const float2 *lpol, 
 #pragma unroll
   for (int ti = 0; ti < kTiers; ++ti) {
     if (!((tiers >> ti) & 1u)) continue;
+    if (exact) {  // the exact-query variant: q / ||q|| itself, for every tier
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int a = 4 * lane + k;
+        const int half = a >> 6, s = a & 63;
+        qt[ti * 2 * QT_HALF + half * QT_HALF + ((s >> 1) * G + g) * 2 + (s & 1)] =
+            qn > 0.0 ? (float)(x[k] / qn) : 0.0f;
+      }
+      continue;
+    }
     int c[4];
     switch (ti) {
       case 0: lane_codes<3>(x, S, x127, lane, pol_c2, az_c2, c); break;
@@ -447,8 +461,10 @@ __device__ __forceinline__ void ada_2page_f(const uint8_t *recA, const uint8_t *
 // 16 pairs of one 16-byte code chunk (32 fields) of both pages, so the loop
 // body (and the instruction footprint) is half of the unrolled one.  The
 // (cos, sin) table of b = 4 is 16 float2 = one 128-byte row starting at a
-// 128-byte aligned shared address: a field's entry address is
-// ((chunk word >> shift) & 0x78) | table.
+// 256-byte aligned shared address.  Each code word is spread once into
+// bytes holding 8 x code (even fields in E, odd fields in O); a field's entry
+// address is then one byte permute: the entry offset as the low byte under
+// the table's upper address bytes.
 template <int G, int QT_HALF>
 __device__ __forceinline__ void ada_2page_f4(const uint8_t *recA, const uint8_t *recB, const float *qt,
                                              uint32_t lpol_s, uint32_t laz_s, int lane, float (&fA)[G],
@@ -476,17 +492,16 @@ __device__ __forceinline__ void ada_2page_f4(const uint8_t *recA, const uint8_t 
 #pragma unroll
       for (int pg = 0; pg < 2; ++pg) {
         const uint32_t w = pg ? WB[pq >> 2] : WA[pq >> 2];
-        const int sh0 = 8 * (pq & 3), sh1 = sh0 + 4;  // bit offsets of the two fields
-        const uint32_t o0 = (sh0 >= 3 ? (w >> (sh0 - 3)) : (w << (3 - sh0))) & 0x78u;
-        const uint32_t o1 = (w >> (sh1 - 3)) & 0x78u;
+        const uint32_t ev = (w << 3) & 0x78787878u, od = (w >> 1) & 0x78787878u;  // CSE'd per word
+        const uint32_t sel = 0x7650u | (uint32_t)(pq & 3);
         float2 e0, e1;
         if (pq == 15) {
-          e0 = lds_f2((tail ? laz_s : lpol_s) | o0);
-          const float2 t1 = lds_f2(lpol_s | o1);
+          e0 = lds_f2(__byte_perm(ev, tail ? laz_s : lpol_s, sel));
+          const float2 t1 = lds_f2(__byte_perm(od, lpol_s, sel));
           e1 = make_float2(tail ? 1.0f : t1.x, tail ? 0.0f : t1.y);
         } else {
-          e0 = lds_f2(lpol_s | o0);
-          e1 = lds_f2(lpol_s | o1);
+          e0 = lds_f2(__byte_perm(ev, lpol_s, sel));
+          e1 = lds_f2(__byte_perm(od, lpol_s, sel));
         }
         const float u0 = Ps[pg] * e0.x, tt = Ps[pg] * e0.y;
         uu[pg] = make_float2(u0, tt * e1.x);
@@ -764,7 +779,8 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
     for (int g = wid; g < G; g += NCW) {
       const uint16_t *qrow = p.q + ((int64_t)b * p.Hq + (int64_t)h * G + g) * kD;
       if constexpr (ADA) {
-        const float qn = ada_qprep_row<G, Ly::QT_HALF>(qrow, g, lpol, laz, pol_c2, az_c2, qt, lane, p.tiers);
+        const float qn = ada_qprep_row<G, Ly::QT_HALF>(qrow, g, lpol, laz, pol_c2, az_c2, qt, lane, p.tiers,
+                                                       (p.flags & SPKV_DECODE_EXACT_Q) != 0u);
         if (lane == 0) sc[g] = qn * kLog2e * 0.08838834764831845f;
       } else {
         dense_qprep_row<G, Ly::QT_HALF>(qrow, g, qt, lane);
@@ -1294,7 +1310,8 @@ __global__ void __launch_bounds__(32) debug_logits_kernel(SplitParams p, float *
   __syncwarp();
   for (int g = 0; g < G; ++g) {
     const float n = ada_qprep_row<G, QT_HALF>(p.q + ((int64_t)b * p.Hq + (int64_t)h * G + g) * kD, g, lpol, laz,
-                                              pol_c2, az_c2, qt, lane, 0xfu);
+                                              pol_c2, az_c2, qt, lane, 0xfu,
+                                              (p.flags & SPKV_DECODE_EXACT_Q) != 0u);
     if (lane == 0) qn[g] = n;
   }
   __syncwarp();
@@ -1459,6 +1476,7 @@ void fill_cache(SplitParams &sp, const spkv_cache *c) {
   sp.keep = c->keep_mask;
   sp.err = c->err_flags;
   sp.tiers = c->tiers ? c->tiers : 0xfu;
+  sp.flags = 0u;
   sp.Hkv = c->num_kv_heads;
   sp.num_pages = c->num_pages;
 }
@@ -1481,15 +1499,17 @@ extern "C" size_t spkv_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv
   return ws_bytes_for(B, Hq, Hkv, C);
 }
 
-extern "C" spkv_status spkv_decode_attention(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t Hq,
-                                             const int32_t *block_table, int32_t max_pages,
-                                             const int32_t *ctx_lens, int32_t max_ctx, void *out,
-                                             int32_t out_is_bf16, void *ws, size_t ws_bytes, int32_t num_splits,
-                                             void *stream) {
+extern "C" spkv_status spkv_decode_attention_ex(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t Hq,
+                                                const int32_t *block_table, int32_t max_pages,
+                                                const int32_t *ctx_lens, int32_t max_ctx, void *out,
+                                                int32_t out_is_bf16, void *ws, size_t ws_bytes, int32_t num_splits,
+                                                uint32_t flags, void *stream) {
+  if (flags & ~SPKV_DECODE_EXACT_Q) return SPKV_ERR_INVALID_ARG;
   spkv_status st = check_cache(cache);
   if (st != SPKV_OK) return st;
   DecodeArgs a;
   fill_cache(a.sp, cache);
+  a.sp.flags = flags;
   st = prep_batch(a.sp, cache->num_kv_heads, q, B, Hq, block_table, max_pages, ctx_lens, max_ctx, out, ws, ws_bytes,
                   num_splits, &a.G, &a.num_splits);
   if (st != SPKV_OK) return st;
@@ -1497,6 +1517,15 @@ extern "C" spkv_status spkv_decode_attention(const spkv_cache *cache, const uint
   a.out = out;
   a.out_bf16 = out_is_bf16 ? 1 : 0;
   return launch_split_and_merge<true>(a, (cudaStream_t)stream);
+}
+
+extern "C" spkv_status spkv_decode_attention(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t Hq,
+                                             const int32_t *block_table, int32_t max_pages,
+                                             const int32_t *ctx_lens, int32_t max_ctx, void *out,
+                                             int32_t out_is_bf16, void *ws, size_t ws_bytes, int32_t num_splits,
+                                             void *stream) {
+  return spkv_decode_attention_ex(cache, q, B, Hq, block_table, max_pages, ctx_lens, max_ctx, out, out_is_bf16, ws,
+                                  ws_bytes, num_splits, 0u, stream);
 }
 
 extern "C" spkv_status spkv_dense_decode(const uint16_t *k_pages, const uint16_t *v_pages, int32_t num_pages,
@@ -1551,9 +1580,10 @@ extern "C" spkv_status spkv_decompress_then_dot(const spkv_cache *cache, uint16_
   return launch_split_and_merge<false>(a, s);
 }
 
-extern "C" spkv_status spkv_debug_logits(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t Hq,
-                                         const int32_t *block_table, int32_t max_pages, const int32_t *ctx_lens,
-                                         int32_t max_ctx, float *logits, void *stream) {
+extern "C" spkv_status spkv_debug_logits_ex(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t Hq,
+                                            const int32_t *block_table, int32_t max_pages, const int32_t *ctx_lens,
+                                            int32_t max_ctx, float *logits, uint32_t flags, void *stream) {
+  if (flags & ~SPKV_DECODE_EXACT_Q) return SPKV_ERR_INVALID_ARG;
   spkv_status st = check_cache(cache);
   if (st != SPKV_OK) return st;
   if (B < 0 || Hq < 1 || max_pages < 0 || max_ctx < 0 || Hq % cache->num_kv_heads) return SPKV_ERR_INVALID_ARG;
@@ -1563,6 +1593,7 @@ extern "C" spkv_status spkv_debug_logits(const spkv_cache *cache, const uint16_t
   if (!q || !block_table || !ctx_lens || !logits || ((uintptr_t)q & 7)) return SPKV_ERR_INVALID_ARG;
   SplitParams sp;
   fill_cache(sp, cache);
+  sp.flags = flags;
   sp.q = q;
   sp.B = B;
   sp.Hq = Hq;
@@ -1582,4 +1613,10 @@ extern "C" spkv_status spkv_debug_logits(const spkv_cache *cache, const uint16_t
     case 8: debug_logits_kernel<8><<<grid, 32, 0, s>>>(sp, logits); break;
   }
   return cudaGetLastError() == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
+}
+
+extern "C" spkv_status spkv_debug_logits(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t Hq,
+                                         const int32_t *block_table, int32_t max_pages, const int32_t *ctx_lens,
+                                         int32_t max_ctx, float *logits, void *stream) {
+  return spkv_debug_logits_ex(cache, q, B, Hq, block_table, max_pages, ctx_lens, max_ctx, logits, 0u, stream);
 }

@@ -10,7 +10,7 @@ import ctypes
 
 import torch
 
-from ._lib import check, lib
+from ._lib import DECODE_EXACT_Q, check, lib
 from .cache import HEAD_DIM, SpkvCache
 
 
@@ -96,16 +96,22 @@ def _ws(ws, B, Hq, Hkv, max_ctx, num_splits, device):
 
 def decode_attention(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tensor, ctx_lens: torch.Tensor,
                      max_ctx: int, out=None, out_dtype=torch.float32, ws=None, num_splits: int = 0,
-                     stream=None) -> torch.Tensor:
-    """spkv_decode_attention: ADA decode straight from the codes; returns out [B, Hq, 128]."""
+                     stream=None, exact_q: bool = False) -> torch.Tensor:
+    """spkv_decode_attention: ADA decode straight from the codes; returns out [B, Hq, 128].
+
+    exact_q=True calls spkv_decode_attention_ex with SPKV_DECODE_EXACT_Q (the
+    unquantised unit query in f_b)."""
     _batch_checks(q, block_table, ctx_lens)
     B, Hq, _ = q.shape
     out = _out_buffer(out, B, Hq, out_dtype, q.device)
     ws, wsb = _ws(ws, B, Hq, cache.num_kv_heads, max_ctx, num_splits, q.device)
     c = cache.c_struct()
-    check(lib.spkv_decode_attention(ctypes.byref(c), _ptr(q), B, Hq, _ptr(block_table), block_table.shape[1],
-                                    _ptr(ctx_lens), int(max_ctx), _ptr(out), int(out.dtype == torch.bfloat16),
-                                    _ptr(ws), wsb, int(num_splits), _stream(stream)), "spkv_decode_attention")
+    args = (ctypes.byref(c), _ptr(q), B, Hq, _ptr(block_table), block_table.shape[1], _ptr(ctx_lens), int(max_ctx),
+            _ptr(out), int(out.dtype == torch.bfloat16), _ptr(ws), wsb, int(num_splits))
+    if exact_q:
+        check(lib.spkv_decode_attention_ex(*args, DECODE_EXACT_Q, _stream(stream)), "spkv_decode_attention_ex")
+    else:
+        check(lib.spkv_decode_attention(*args, _stream(stream)), "spkv_decode_attention")
     return out
 
 
@@ -164,12 +170,13 @@ def decompress_then_dot(cache: SpkvCache, k_scratch: torch.Tensor, q: torch.Tens
 
 
 def debug_logits(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tensor, ctx_lens: torch.Tensor,
-                 max_ctx: int, stream=None) -> torch.Tensor:
-    """spkv_debug_logits: ADA logits [B, Hq, max_ctx] fp32 (NaN where not written)."""
+                 max_ctx: int, stream=None, exact_q: bool = False) -> torch.Tensor:
+    """spkv_debug_logits(_ex): ADA logits [B, Hq, max_ctx] fp32 (NaN where not written)."""
     _batch_checks(q, block_table, ctx_lens)
     B, Hq, _ = q.shape
     logits = torch.full((B, Hq, max(max_ctx, 1)), float("nan"), dtype=torch.float32, device=q.device)
     c = cache.c_struct()
-    check(lib.spkv_debug_logits(ctypes.byref(c), _ptr(q), B, Hq, _ptr(block_table), block_table.shape[1],
-                                _ptr(ctx_lens), int(max_ctx), _ptr(logits), _stream(stream)), "spkv_debug_logits")
+    check(lib.spkv_debug_logits_ex(ctypes.byref(c), _ptr(q), B, Hq, _ptr(block_table), block_table.shape[1],
+                                   _ptr(ctx_lens), int(max_ctx), _ptr(logits), DECODE_EXACT_Q if exact_q else 0,
+                                   _stream(stream)), "spkv_debug_logits_ex")
     return logits

@@ -162,6 +162,22 @@ SPKV_API spkv_status spkv_decode_attention(const spkv_cache *cache, const uint16
                                   int32_t max_ctx, void *out, int32_t out_is_bf16, void *ws, size_t ws_bytes,
                                   int32_t num_splits, void *stream);
 
+/* Flag bits of spkv_decode_attention_ex and spkv_debug_logits_ex. */
+#define SPKV_DECODE_EXACT_Q 1u
+
+/* spkv_decode_attention with flag bits; flags = 0 is spkv_decode_attention.
+ *   SPKV_DECODE_EXACT_Q  the exact-query variant of f_b.  Section 2.1 of the
+ *       summary writes f_b(c_q, c_k), a cosine from the codes of both sides,
+ *       and leaves f_b itself open; with this flag the query is NOT coded:
+ *       f = <q / ||q||, u~(c_k)>, the unquantised unit query against the
+ *       decoded key (a zero query gives f = 0).  Same bytes read per token.
+ * Unknown flag bits: SPKV_ERR_INVALID_ARG (before any launch).  Every other
+ * argument, layout and rule is that of spkv_decode_attention. */
+SPKV_API spkv_status spkv_decode_attention_ex(const spkv_cache *cache, const uint16_t *q, int32_t B,
+                                     int32_t num_q_heads, const int32_t *block_table, int32_t max_pages,
+                                     const int32_t *ctx_lens, int32_t max_ctx, void *out, int32_t out_is_bf16,
+                                     void *ws, size_t ws_bytes, int32_t num_splits, uint32_t flags, void *stream);
+
 /* Dense paged decode over bf16 keys, the uncompressed comparison path
  * (section 4 of the summary compares against dense KV):
  * logit = q . k / sqrt(128), same paging, mask, split and output rules as
@@ -222,6 +238,12 @@ SPKV_API spkv_status spkv_decode_attention_static_ws(const spkv_cache *cache, co
 SPKV_API spkv_status spkv_debug_logits(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t num_q_heads,
                               const int32_t *block_table, int32_t max_pages, const int32_t *ctx_lens,
                               int32_t max_ctx, float *logits, void *stream);
+
+/* spkv_debug_logits with the flag bits of spkv_decode_attention_ex. */
+SPKV_API spkv_status spkv_debug_logits_ex(const spkv_cache *cache, const uint16_t *q, int32_t B,
+                                 int32_t num_q_heads, const int32_t *block_table, int32_t max_pages,
+                                 const int32_t *ctx_lens, int32_t max_ctx, float *logits, uint32_t flags,
+                                 void *stream);
 
 #ifdef __cplusplus
 }

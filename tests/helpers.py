@@ -55,14 +55,18 @@ def near_integer(pos: np.ndarray, rel: float = 1e-12) -> np.ndarray:
     return d <= rel * np.maximum(1.0, np.abs(np.where(fin, pos, 0.0)))
 
 
-def oracle_seq(wl, b: int, h: int, want_logits: bool = False):
+def oracle_seq(wl, b: int, h: int, want_logits: bool = False, exact_q: bool = False):
     """Oracle ADA output for the G query heads of (b, h), encoding the keys itself."""
     keys = wl.keys_bits(b, h)
     bits = wl.token_bits(b)
     L, D = float(wl.rad_lo[h]), float(wl.rad_step[h])
     codes, rcode = oracle.encode(keys, bits, L, D)
     return oracle.ada_group(wl.q_bits(b, h), codes, bits, rcode, L, D, wl.values_bits(b, h), keep=wl.keep_of(b),
-                            want_logits=want_logits)
+                            want_logits=want_logits, exact_q=exact_q)
+
+
+def oracle_seq_exact_q(wl, b: int, h: int):
+    return oracle_seq(wl, b, h, exact_q=True)
 
 
 def oracle_seq_dense(wl, b: int, h: int):

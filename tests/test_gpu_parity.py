@@ -158,6 +158,36 @@ def test_debug_logits_parity(spkv):
         assert d.max() <= FB_TOL, d.max()
 
 
+def test_exact_query_decode_parity(spkv):
+    """The exact-query variant (SPKV_DECODE_EXACT_Q) against the oracle's,
+    mixed tiers, mask and ragged lengths; and its logits to |d f_b| <= 1e-4."""
+    m = spkv[0]
+    wl, cache = _build(spkv, RAGGED, B=4, ctx=[2000, 333, 17, 4100], Hq=8, Hkv=2)
+    out = _decode(spkv, wl, cache, exact_q=True).cpu().numpy()
+    err = helpers.max_abs_diff_groups(out, wl, helpers.all_groups(wl), helpers.oracle_seq_exact_q)
+    assert err <= OUT_TOL, err
+    lg = m.debug_logits(cache, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx, exact_q=True).cpu().numpy()
+    for b, h in helpers.all_groups(wl):
+        n = int(wl.ctx[b])
+        _, ref = helpers.oracle_seq(wl, b, h, want_logits=True, exact_q=True)
+        keys, bits = wl.keys_bits(b, h), wl.token_bits(b)
+        _, rc = oracle.encode(keys, bits, float(wl.rad_lo[h]), float(wl.rad_step[h]))
+        scale = helpers.logit_scale(wl, b, h, rc)
+        got = lg[b, h * wl.G:(h + 1) * wl.G, :n].astype(np.float64)
+        ev = np.isinf(ref)
+        assert np.array_equal(np.isinf(got), ev)
+        d = np.abs(got[~ev] - ref[~ev]) / scale[~ev]
+        assert d.max() <= FB_TOL, d.max()
+
+
+def test_exact_query_decode_parity_b4_pairs(spkv):
+    """Exact query on an all-b=4 cache (the narrow ring and the paired b = 4 loop), G = 4."""
+    wl, cache = _build(spkv, LLAMA, B=2, ctx=[1000, 2049])
+    out = _decode(spkv, wl, cache, exact_q=True).cpu().numpy()
+    err = helpers.max_abs_diff_groups(out, wl, helpers.all_groups(wl), helpers.oracle_seq_exact_q)
+    assert err <= OUT_TOL, err
+
+
 def _reorder_tol(wl):
     # A different split count changes only the fp32 summation order and the
     # running maxima at which p is split into bf16 hi + lo parts for the

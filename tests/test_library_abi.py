@@ -69,6 +69,13 @@ def test_host_argument_checks(lib):
     assert _decode(m, _fake_cache(m), ws_bytes=16) == 3    # workspace too small
     assert _decode(m, _fake_cache(m), B=5000) == 2         # batch beyond the supported maximum
     assert _decode(m, _fake_cache(m), B=0) == 0            # empty batch: nothing to do
+    # flags: unknown bits are rejected before anything else; known bits pass the checks
+    c = _fake_cache(m)
+    assert L.spkv_decode_attention_ex(ctypes.byref(c), 0x1000, 0, 8, 0x2000, 4, 0x3000, 64, 0x4000, 0, 0x5000,
+                                      1 << 20, 0, 2, None) == 1
+    assert L.spkv_decode_attention_ex(ctypes.byref(c), 0x1000, 0, 8, 0x2000, 4, 0x3000, 64, 0x4000, 0, 0x5000,
+                                      1 << 20, 1, 1, None) == 0  # empty batch, one split: no device query
+    assert L.spkv_debug_logits_ex(ctypes.byref(c), 0x1000, 1, 8, 0x2000, 4, 0x3000, 64, 0x4000, 4, None) == 1
     # encode: negative sizes / misaligned keys
     c = _fake_cache(m)
     assert L.spkv_encode_keys(ctypes.byref(c), 0x1000, None, 0x2000, -1, 1, 0x3000, 4, None) == 1
