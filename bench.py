@@ -1,10 +1,10 @@
 #!/usr/bin/env python
 """Benchmark: ADA paged decode KV tokens/s on B200 (one JSON line on rank 0).
 
-One step = the whole decode hot path for one batch: append the step's new
-token (key and value) of every sequence through spkv_encode_keys, then
-spkv_decode_attention over all ctx tokens of every sequence (split kernel +
-merge kernel).  Default workload: Llama-3-8B-shaped layer decode, B = 8,
+One step = the whole decode hot path for one batch, in one library call
+(spkv_decode_attention_append): append the step's new token (key and value)
+of every sequence into its page, then decode over all ctx tokens of every
+sequence (split kernel with the fused append + merge kernel).  Default workload: Llama-3-8B-shaped layer decode, B = 8,
 32 query / 8 kv heads, d = 128, ctx = 32768, page 16, b = 4 (673 MB of codes,
 radii and values per step: far larger than the 126 MB L2, so no flush is
 needed between steps).
@@ -170,14 +170,13 @@ def run_spkv(args, rank, world, local):
     # the step's new token: the last context position of every sequence
     last = torch.as_tensor((wl.ctx - 1).astype(np.int32), device=dev)
     new_idx = torch.as_tensor(wl.seq_off[1:] - 1, device=dev).long()
-    new_k = wl.keys[new_idx].unsqueeze(1).contiguous()     # [B, 1, Hkv, 128]
-    new_v = wl.values[new_idx].unsqueeze(1).contiguous()
+    new_k = wl.keys[new_idx].contiguous()     # [B, Hkv, 128]
+    new_v = wl.values[new_idx].contiguous()
     stream = torch.cuda.current_stream(dev)
 
     def step(q, k, v, o):
-        spkv.encode_keys(cache, k, last, wl.block_table, values=v, stream=stream)
-        spkv.decode_attention(cache, q, wl.block_table, ctx, max_ctx, out=o, ws=ws, num_splits=splits,
-                              stream=stream)
+        spkv.decode_attention_append(cache, k, v, q, wl.block_table, ctx, max_ctx, out=o, ws=ws,
+                                     num_splits=splits, stream=stream)
 
     for _ in range(args.warmup):
         step(wl.q, new_k, new_v, out)
@@ -195,10 +194,9 @@ def run_spkv(args, rank, world, local):
     with ClockSampler(local) as clk:
         t_start.record(stream)
         for i in range(args.steps):
-            spkv.encode_keys(cache, new_k, last, wl.block_table, values=new_v, stream=stream)
             ev_dec[i][0].record(stream)
-            spkv.decode_attention(cache, wl.q, wl.block_table, ctx, max_ctx, out=out, ws=ws, num_splits=splits,
-                                  stream=stream)
+            spkv.decode_attention_append(cache, new_k, new_v, wl.q, wl.block_table, ctx, max_ctx, out=out, ws=ws,
+                                         num_splits=splits, stream=stream)
             ev_dec[i][1].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
@@ -265,15 +263,15 @@ def run_spkv(args, rank, world, local):
                        "page": 16, "bits": sorted(set(int(b) for b in wl.page_bits)), "splits": splits,
                        "kv_tokens_per_step": tokens, "algorithmic_bytes_per_step": bytes_step,
                        "l2": "no flush: the step streams %.0f MB > 126 MB L2" % (bytes_step / 1e6),
-                       "step": "append 1 token/sequence (spkv_encode_keys) + spkv_decode_attention",
+                       "step": "spkv_decode_attention_append: append 1 token/sequence + decode, one call",
                        "parallelism": f"dp{world} (independent batches)"},
-            "roofline": {"bound": "hbm", "kernel": "spkv_decode_attention (split + merge kernels)",
+            "roofline": {"bound": "hbm", "kernel": "spkv_decode_attention_append (split kernel with the append + merge)",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS,
                          "traffic": traffic, "decode_ms": dec_ms},
             "e2e": {"value": whole_job_rate(tokens, world, e2e_ms), "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": 2 * args.steps,
             "clocks": clocks,
         }
         if extras:
@@ -309,6 +307,18 @@ def compare_paths(args, spkv, workload, wl, cache, ctx, max_ctx, splits, ws, str
     ada_ms = timeit(lambda: spkv.decode_attention(cache, wl.q, wl.block_table, ctx, max_ctx, ws=ws,
                                                   num_splits=splits, stream=stream))
     res["ada_decode_ms"] = ada_ms
+    # the step as two calls (spkv_encode_keys + spkv_decode_attention) vs the fused append
+    last = (ctx - 1).to(torch.int32)
+    idx = torch.as_tensor(wl.seq_off[1:] - 1, device=dev).long()
+    nk, nv = wl.keys[idx].contiguous(), wl.values[idx].contiguous()
+
+    def two_calls():
+        spkv.encode_keys(cache, nk.unsqueeze(1), last, wl.block_table, values=nv.unsqueeze(1), stream=stream)
+        spkv.decode_attention(cache, wl.q, wl.block_table, ctx, max_ctx, ws=ws, num_splits=splits, stream=stream)
+
+    res["step_two_calls_ms"] = timeit(two_calls)
+    res["step_fused_append_ms"] = timeit(lambda: spkv.decode_attention_append(
+        cache, nk, nv, wl.q, wl.block_table, ctx, max_ctx, ws=ws, num_splits=splits, stream=stream))
     kp, vp = workload.dense_pages(wl)
     dense_ms = timeit(lambda: spkv.dense_decode(kp, vp, wl.q, wl.block_table, ctx, max_ctx, ws=ws,
                                                 num_splits=splits, stream=stream))

@@ -7,5 +7,6 @@ loudly when the CUDA library has not been built.
 """
 from ._lib import LIB_PATH, SpkvError, lib  # noqa: F401
 from .cache import SpkvCache  # noqa: F401
-from .ops import (alloc_workspace, debug_logits, decode_attention, decode_attention_static_ws,  # noqa: F401
-                  decompress_then_dot, default_splits, dense_decode, encode_keys, workspace_bytes)
+from .ops import (alloc_workspace, debug_logits, decode_attention, decode_attention_append,  # noqa: F401
+                  decode_attention_static_ws, decompress_then_dot, default_splits, dense_decode, encode_keys,
+                  workspace_bytes)

@@ -36,7 +36,7 @@
 
 #include <type_traits>
 
-#include "spkv_common.cuh"
+#include "spkv_encode.cuh"
 
 namespace spkv {
 
@@ -160,7 +160,10 @@ struct Layout {
   static constexpr int off_bar = off_sc + ((G + 2) * 4 + 15) / 16 * 16;  // full, empty, value slots
   static constexpr int off_meta = off_bar + (2 * NST + 2 * NCW) * 8;
   static constexpr int off_misc = off_meta + NST * 32;            // abort flag + scan scratch
-  static constexpr int off_P = off_misc + 16 + 36 * 4;
+  // the producer's own fp64 edge tables and code scratch (fused append)
+  static constexpr int off_pe = (off_misc + 16 + 36 * 4 + 15) / 16 * 16;
+  static constexpr int pe_bytes = ADA ? 2 * kLutEntries * 8 + 128 : 0;
+  static constexpr int off_P = off_pe + pe_bytes;
   // + 1024 bytes of slack to align the carve-up base to 1024
   static constexpr size_t bytes(int B) { return (size_t)off_P + (size_t)(B + 1) * 4 + 16 + 1024; }
   // two CTAs per SM: 228 KB of shared memory minus 1 KB reserved per CTA
@@ -178,6 +181,10 @@ struct SplitParams {
   uint32_t *err;
   uint32_t tiers;  // tiers the query is coded for (bit t: b = {3,4,6,8}[t])
   uint32_t flags;  // SPKV_DECODE_* bits
+  // fused single-token append (ADA only): the key and value [B, H_kv, 128] of
+  // each sequence's token ctx - 1, encoded into its page before it is read;
+  // nullptr: no append
+  const uint16_t *new_k, *new_v;
   int Hkv, num_pages;
   const uint16_t *q;
   int B, Hq;
@@ -586,6 +593,25 @@ __device__ __forceinline__ void dense_page_logits(const uint8_t *kpage, const fl
 // the path); m is in log2 units.
 constexpr int kPartial = 132;
 
+// Fused single-token append, by the producer warp: the new key of kv row
+// (b, h) -- token ctx_lens[b] - 1, the last one of the row's last page pid,
+// whose record (width `bits`) starts at byte rec_off of the arena -- is
+// encoded into its slot exactly as spkv_encode_keys would write it, and the
+// new value row goes to the same slot of the value page.  Called before the
+// page's copy is issued; the caller fences the stores for the async proxy.
+__device__ __noinline__ void append_token(const SplitParams &p, int b, int h, int pid, int bits, uint64_t rec_off,
+                                          const double *pol_c2, const double *az_c2, uint8_t *codes_smem,
+                                          int lane) {
+  const int slot = (p.ctx_lens[b] - 1) % kPage;
+  const int64_t row = (int64_t)b * p.Hkv + h;
+  encode_key_warp(p.new_k + row * kD, bits, const_cast<uint8_t *>(p.arena) + rec_off, slot, p.rad_lo[h],
+                  p.rad_step[h], pol_c2, az_c2, codes_smem, lane, p.err);
+  const uint2 v = *reinterpret_cast<const uint2 *>(p.new_v + row * kD + 4 * lane);
+  *reinterpret_cast<uint2 *>(const_cast<uint16_t *>(p.v_pages) + (((int64_t)pid * p.Hkv + h) * kPage + slot) * kD +
+                             4 * lane) = v;
+  __syncwarp();
+}
+
 template <bool ADA, int G, bool NW>
 __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
     split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap vmap) {
@@ -600,6 +626,9 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
   float *qt = reinterpret_cast<float *>(smem + Ly::off_qt);
   double *pol_c2 = reinterpret_cast<double *>(smem + Ly::off_pbc2);
   double *az_c2 = pol_c2 + kLutEntries;
+  double *pe_pol = reinterpret_cast<double *>(smem + Ly::off_pe);  // producer's edge tables
+  double *pe_az = pe_pol + kLutEntries;
+  uint8_t *pe_codes = smem + Ly::off_pe + 2 * kLutEntries * 8;
   float *pbuf_all = reinterpret_cast<float *>(smem + Ly::off_pbc2);
   float *sc = reinterpret_cast<float *>(smem + Ly::off_sc);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + Ly::off_bar);
@@ -641,7 +670,7 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
     // units is fetched by the 32 lanes in two dependent rounds (block table,
     // then header / mask), half a batch ahead.
     struct A_ {
-      int pid, ntok, h, ok;
+      int pid, ntok, h, ok, last, b;
     };
     struct B_ {
       uint32_t off16;
@@ -649,7 +678,7 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
       uint32_t keep;
     };
     auto phaseA = [&](int kb) -> A_ {
-      A_ a{0, 0, 0, 0};
+      A_ a{0, 0, 0, 0, 0, 0};
       const int k = kb + lane;
       if (k < n_units) {
         const int64_t u = u0 + k;
@@ -661,6 +690,8 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
         a.pid = p.block_table[(int64_t)b * p.max_pages + j];
         const int ctx = p.ctx_lens[b];
         a.ntok = min(kPage, ctx - j * kPage);
+        a.last = j == np - 1;
+        a.b = b;
         a.ok = 1;
       }
       return a;
@@ -677,6 +708,7 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
       }
       return r;
     };
+    bool pe_built = false;  // the producer's edge tables (built on the first append)
     A_ an = phaseA(0);
     B_ bn = phaseB(an);
     int k_last = -1;
@@ -712,6 +744,28 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
         if (i0 == 16) bn = phaseB(an);
         const int k = kb + lane, s = k % NST, r = k / NST;
         const bool mine = lane >= i0 && lane < i0 + kIssue && lane < cnt;
+        if constexpr (ADA) {
+          // fused append: a row's last page gets the step's token before its copy
+          uint32_t todo = p.new_k ? __ballot_sync(0xffffffffu, mine && valid && ac.last) : 0u;
+          if (todo) {
+            if (!pe_built) {
+              build_edge_tables(pe_pol, pe_az, lane, 32);
+              __syncwarp();
+              pe_built = true;
+            }
+            while (todo) {
+              const int src = __ffs(todo) - 1;
+              todo &= todo - 1;
+              append_token(p, __shfl_sync(0xffffffffu, ac.b, src), __shfl_sync(0xffffffffu, ac.h, src),
+                           __shfl_sync(0xffffffffu, ac.pid, src), __shfl_sync(0xffffffffu, bc.bits, src),
+                           __shfl_sync(0xffffffffu, rec_off, src), pe_pol, pe_az, pe_codes, lane);
+            }
+            // the copies below (and the consumers' value TMA) read what was written
+            __threadfence();
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __syncwarp();
+          }
+        }
         if (mine) {
           if (r > 0) mbar_wait_sleepy(&empty[s], (uint32_t)(r - 1) & 1u, abort_flag, p.err);
           StageMeta m;
@@ -1477,6 +1531,8 @@ void fill_cache(SplitParams &sp, const spkv_cache *c) {
   sp.err = c->err_flags;
   sp.tiers = c->tiers ? c->tiers : 0xfu;
   sp.flags = 0u;
+  sp.new_k = nullptr;
+  sp.new_v = nullptr;
   sp.Hkv = c->num_kv_heads;
   sp.num_pages = c->num_pages;
 }
@@ -1499,17 +1555,20 @@ extern "C" size_t spkv_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv
   return ws_bytes_for(B, Hq, Hkv, C);
 }
 
-extern "C" spkv_status spkv_decode_attention_ex(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t Hq,
-                                                const int32_t *block_table, int32_t max_pages,
-                                                const int32_t *ctx_lens, int32_t max_ctx, void *out,
-                                                int32_t out_is_bf16, void *ws, size_t ws_bytes, int32_t num_splits,
-                                                uint32_t flags, void *stream) {
+namespace spkv {
+namespace {
+spkv_status decode_ada(const spkv_cache *cache, const uint16_t *new_k, const uint16_t *new_v, const uint16_t *q,
+                       int32_t B, int32_t Hq, const int32_t *block_table, int32_t max_pages, const int32_t *ctx_lens,
+                       int32_t max_ctx, void *out, int32_t out_is_bf16, void *ws, size_t ws_bytes,
+                       int32_t num_splits, uint32_t flags, void *stream) {
   if (flags & ~SPKV_DECODE_EXACT_Q) return SPKV_ERR_INVALID_ARG;
   spkv_status st = check_cache(cache);
   if (st != SPKV_OK) return st;
   DecodeArgs a;
   fill_cache(a.sp, cache);
   a.sp.flags = flags;
+  a.sp.new_k = new_k;
+  a.sp.new_v = new_v;
   st = prep_batch(a.sp, cache->num_kv_heads, q, B, Hq, block_table, max_pages, ctx_lens, max_ctx, out, ws, ws_bytes,
                   num_splits, &a.G, &a.num_splits);
   if (st != SPKV_OK) return st;
@@ -1517,6 +1576,29 @@ extern "C" spkv_status spkv_decode_attention_ex(const spkv_cache *cache, const u
   a.out = out;
   a.out_bf16 = out_is_bf16 ? 1 : 0;
   return launch_split_and_merge<true>(a, (cudaStream_t)stream);
+}
+}  // namespace
+}  // namespace spkv
+
+extern "C" spkv_status spkv_decode_attention_ex(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t Hq,
+                                                const int32_t *block_table, int32_t max_pages,
+                                                const int32_t *ctx_lens, int32_t max_ctx, void *out,
+                                                int32_t out_is_bf16, void *ws, size_t ws_bytes, int32_t num_splits,
+                                                uint32_t flags, void *stream) {
+  return decode_ada(cache, nullptr, nullptr, q, B, Hq, block_table, max_pages, ctx_lens, max_ctx, out, out_is_bf16,
+                    ws, ws_bytes, num_splits, flags, stream);
+}
+
+extern "C" spkv_status spkv_decode_attention_append(const spkv_cache *cache, const uint16_t *new_keys,
+                                                    const uint16_t *new_values, const uint16_t *q, int32_t B,
+                                                    int32_t Hq, const int32_t *block_table, int32_t max_pages,
+                                                    const int32_t *ctx_lens, int32_t max_ctx, void *out,
+                                                    int32_t out_is_bf16, void *ws, size_t ws_bytes,
+                                                    int32_t num_splits, uint32_t flags, void *stream) {
+  if (B > 0 && (!new_keys || !new_values)) return SPKV_ERR_INVALID_ARG;
+  if (((uintptr_t)new_keys & 7) || ((uintptr_t)new_values & 7)) return SPKV_ERR_INVALID_ARG;
+  return decode_ada(cache, new_keys, new_values, q, B, Hq, block_table, max_pages, ctx_lens, max_ctx, out,
+                    out_is_bf16, ws, ws_bytes, num_splits, flags, stream);
 }
 
 extern "C" spkv_status spkv_decode_attention(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t Hq,

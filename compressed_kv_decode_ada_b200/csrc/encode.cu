@@ -16,7 +16,7 @@
 // clamped to 2^b - 1 -- ties go to the upper cell.  The azimuth (angle 127,
 // range [0, 2 pi)) uses the same test on (x_126, x_127) with the half-plane
 // given by the sign of x_127.  The radius code uses fp64 log2.
-#include "spkv_common.cuh"
+#include "spkv_encode.cuh"
 
 namespace spkv {
 namespace {
@@ -43,20 +43,6 @@ struct EncodeSmem {
   double az_c2[kLutEntries];
   uint8_t codes[kEncWarps][128];
 };
-
-// Word w (32 bits) of a slot's bitstream, from the byte-per-angle codes.
-template <int BITS>
-__device__ __forceinline__ uint32_t pack_word(const uint8_t *codes, int w) {
-  const int lo_bit = 32 * w;
-  const int a0 = lo_bit / BITS, a1 = min(127, (lo_bit + 31) / BITS);
-  uint32_t v = 0;
-  for (int a = a0; a <= a1; ++a) {
-    const int sh = a * BITS - lo_bit;
-    const uint32_t c = codes[a];
-    v |= sh >= 0 ? (c << sh) : (c >> (-sh));
-  }
-  return v;
-}
 
 __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams p) {
   __shared__ EncodeSmem sm;
@@ -93,50 +79,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams 
     }
     const int slot = pos % kPage;
 
-    // ---- load x (4 per lane); exact squares and suffix sums in fp64
-    const uint2 raw = *reinterpret_cast<const uint2 *>(p.keys + item * kD + 4 * lane);
-    double x[4], S[4];
-    lane_suffix_sums(raw, lane, x, S);
-    const double x127 = __shfl_sync(0xffffffffu, x[3], 31);
-
-    // ---- angle codes (fp64 decisions), one byte per angle in shared memory
-    uint8_t *codes = sm.codes[wid];
-    int c4[4];
-    switch (bits) {
-      case 3: lane_codes<3>(x, S, x127, lane, sm.pol_c2, sm.az_c2, c4); break;
-      case 4: lane_codes<4>(x, S, x127, lane, sm.pol_c2, sm.az_c2, c4); break;
-      case 6: lane_codes<6>(x, S, x127, lane, sm.pol_c2, sm.az_c2, c4); break;
-      default: lane_codes<8>(x, S, x127, lane, sm.pol_c2, sm.az_c2, c4); break;
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) codes[4 * lane + k] = (uint8_t)c4[k];
-    __syncwarp();
-
-    // ---- pack: lane w < 4b builds word w; store chunk-major
-    uint8_t *recp = p.arena + rec;
-    if (lane < 4 * bits) {
-      uint32_t word;
-      switch (bits) {
-        case 3: word = pack_word<3>(codes, lane); break;
-        case 4: word = pack_word<4>(codes, lane); break;
-        case 6: word = pack_word<6>(codes, lane); break;
-        default: word = pack_word<8>(codes, lane); break;
-      }
-      const int chunk = lane >> 2, wic = lane & 3;
-      *reinterpret_cast<uint32_t *>(recp + (chunk * 16 + slot) * 16 + wic * 4) = word;
-    }
-    // ---- radius code (lane 0 holds S_0 = ||k||^2)
-    if (lane == 0) {
-      const float Lf = p.rad_lo[h], Df = p.rad_step[h];
-      int c = 0;
-      if (!(Df > 0.0f) || !isfinite(Df) || !isfinite(Lf)) {
-        set_err(p.err, SPKV_DEVERR_RADIUS);
-      } else if (S[0] > 0.0) {
-        const double t = (log2(sqrt(S[0])) - (double)Lf) / (double)Df + 0.5;
-        c = t <= 0.0 ? 0 : t >= 255.0 ? 255 : (int)floor(t);
-      }
-      recp[256 * bits + slot] = (uint8_t)c;
-    }
+    encode_key_warp(p.keys + item * kD, bits, p.arena + rec, slot, p.rad_lo[h], p.rad_step[h], sm.pol_c2, sm.az_c2,
+                    sm.codes[wid], lane, p.err);
     // ---- value row (optional)
     if (p.values) {
       const uint2 v = *reinterpret_cast<const uint2 *>(p.values + item * kD + 4 * lane);

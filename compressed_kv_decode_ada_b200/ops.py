@@ -115,6 +115,30 @@ def decode_attention(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tenso
     return out
 
 
+def decode_attention_append(cache: SpkvCache, new_keys: torch.Tensor, new_values: torch.Tensor, q: torch.Tensor,
+                            block_table: torch.Tensor, ctx_lens: torch.Tensor, max_ctx: int, out=None,
+                            out_dtype=torch.float32, ws=None, num_splits: int = 0, stream=None,
+                            exact_q: bool = False) -> torch.Tensor:
+    """spkv_decode_attention_append: write token ctx_lens[b] - 1 of every sequence
+    (new_keys / new_values [B, H_kv, 128] bf16) into its page, then decode over
+    ctx_lens[b] tokens, in the decode's own launches."""
+    _batch_checks(q, block_table, ctx_lens)
+    B, Hq, _ = q.shape
+    for t, name in ((new_keys, "new_keys"), (new_values, "new_values")):
+        _need(t, torch.bfloat16, name, 3)
+        if tuple(t.shape) != (B, cache.num_kv_heads, HEAD_DIM):
+            raise ValueError(f"{name} must be [B, H_kv, 128]")
+    out = _out_buffer(out, B, Hq, out_dtype, q.device)
+    ws, wsb = _ws(ws, B, Hq, cache.num_kv_heads, max_ctx, num_splits, q.device)
+    c = cache.c_struct()
+    check(lib.spkv_decode_attention_append(ctypes.byref(c), _ptr(new_keys), _ptr(new_values), _ptr(q), B, Hq,
+                                           _ptr(block_table), block_table.shape[1], _ptr(ctx_lens), int(max_ctx),
+                                           _ptr(out), int(out.dtype == torch.bfloat16), _ptr(ws), wsb,
+                                           int(num_splits), DECODE_EXACT_Q if exact_q else 0, _stream(stream)),
+          "spkv_decode_attention_append")
+    return out
+
+
 def decode_attention_static_ws(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tensor,
                                ctx_lens: torch.Tensor, max_ctx: int, out=None, out_dtype=torch.float32,
                                num_splits: int = 0, stream=None) -> torch.Tensor:

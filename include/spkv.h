@@ -178,6 +178,30 @@ SPKV_API spkv_status spkv_decode_attention_ex(const spkv_cache *cache, const uin
                                      const int32_t *ctx_lens, int32_t max_ctx, void *out, int32_t out_is_bf16,
                                      void *ws, size_t ws_bytes, int32_t num_splits, uint32_t flags, void *stream);
 
+/* Decode step with the fused single-token append (the serving loop's per-step
+ * path; section 2.3 of the summary maps each new key to its spherical codes
+ * and stores it in the compressed format): for every sequence b with
+ * ctx_lens[b] >= 1 whose pages the decode walks, token ctx_lens[b] - 1 takes
+ *   new_keys[b, h, :]   -> its radius and angle codes, written into slot
+ *                          (ctx - 1) mod 16 of page block_table[b][(ctx - 1) / 16]
+ *                          exactly as spkv_encode_keys writes them, and
+ *   new_values[b, h, :] -> the same slot of v_pages,
+ * for every kv head h, and then the decode of spkv_decode_attention_ex runs
+ * over ctx_lens[b] tokens including it -- all in the decode's own launches
+ * (no separate encode launch).  The result equals spkv_encode_keys with
+ * start_pos = ctx_lens - 1 and n_new = 1 followed by spkv_decode_attention_ex.
+ *   new_keys, new_values  [B, H_kv, 128] bf16, device, 8-byte aligned
+ * Everything else as spkv_decode_attention_ex (flags included).  The page's
+ * header must already hold its bit width; a bad page id / header / record is
+ * flagged by the decode and the token is not written.  Sequences the decode
+ * skips (ctx 0, or ctx > max_ctx: SPKV_DEVERR_CTX) get no append. */
+SPKV_API spkv_status spkv_decode_attention_append(const spkv_cache *cache, const uint16_t *new_keys,
+                                         const uint16_t *new_values, const uint16_t *q, int32_t B,
+                                         int32_t num_q_heads, const int32_t *block_table, int32_t max_pages,
+                                         const int32_t *ctx_lens, int32_t max_ctx, void *out,
+                                         int32_t out_is_bf16, void *ws, size_t ws_bytes, int32_t num_splits,
+                                         uint32_t flags, void *stream);
+
 /* Dense paged decode over bf16 keys, the uncompressed comparison path
  * (section 4 of the summary compares against dense KV):
  * logit = q . k / sqrt(128), same paging, mask, split and output rules as

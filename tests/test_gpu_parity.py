@@ -112,6 +112,59 @@ def test_encode_append_in_steps_matches_one_shot(spkv):
     assert torch.equal(cache2.v_pages, cache.v_pages)
 
 
+def _last_tokens(wl):
+    idx = torch.tensor([int(wl.seq_off[b]) + int(wl.ctx[b]) - 1 for b in range(wl.B)], device=wl.keys.device)
+    return wl.keys[idx].contiguous(), wl.values[idx].contiguous()
+
+
+@pytest.mark.parametrize("cfg,kw", [
+    (RAGGED, dict(B=4, ctx=[37, 1, 2049, 700])),        # mixed tiers, mask, a one-token sequence (wide ring)
+    (LLAMA, dict(B=3, ctx=[16, 1000, 4097])),           # b = 4 only (narrow ring), page-aligned and ragged ends
+])
+def test_fused_append_equals_encode_then_decode(spkv, cfg, kw):
+    """spkv_decode_attention_append writes token ctx - 1 exactly as spkv_encode_keys
+    does (over junk left in the slot) and returns the same output as the two-call path."""
+    m = spkv[0]
+    wl, cache = _build(spkv, cfg, **kw)
+    ref_out = _decode(spkv, wl, cache)
+    ref_arena, ref_v = cache.arena.clone(), cache.v_pages.clone()
+    new_k, new_v = _last_tokens(wl)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    junk_k = torch.randn(new_k.shape, generator=g, device="cuda").to(torch.bfloat16)
+    junk_v = torch.randn(new_v.shape, generator=g, device="cuda").to(torch.bfloat16)
+    last = (wl.ctx_tensor() - 1).to(torch.int32)
+    m.encode_keys(cache, junk_k.unsqueeze(1).contiguous(), last, wl.block_table, values=junk_v.unsqueeze(1).contiguous())
+    torch.cuda.synchronize()
+    assert not torch.equal(cache.arena, ref_arena)
+    out = m.decode_attention_append(cache, new_k, new_v, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx)
+    torch.cuda.synchronize()
+    assert cache.error_flags() == 0
+    assert torch.equal(cache.arena, ref_arena)
+    assert torch.equal(cache.v_pages, ref_v)
+    assert torch.equal(out, ref_out)
+
+
+def test_fused_append_oracle_parity_exact_query(spkv):
+    """The fused append with the exact-query flag against the oracle, from a cache
+    whose last tokens were never encoded."""
+    m, synthetic, workload = spkv
+    wl = synthetic.make_workload(RAGGED, device="cuda", B=3, ctx=[300, 17, 1500], Hq=8, Hkv=2)
+    cache = m.SpkvCache(wl.num_pages, wl.Hkv, wl.page_bits, wl.rad_lo, wl.rad_step, keep_mask=wl.keep_mask)
+    for b in range(wl.B):  # prefill all but the last token of every sequence
+        s, n = int(wl.seq_off[b]), int(wl.ctx[b])
+        if n > 1:
+            m.encode_keys(cache, wl.keys[s:s + n - 1].unsqueeze(0).contiguous(),
+                          torch.zeros(1, dtype=torch.int32, device="cuda"), wl.block_table[b:b + 1].contiguous(),
+                          values=wl.values[s:s + n - 1].unsqueeze(0).contiguous())
+    new_k, new_v = _last_tokens(wl)
+    out = m.decode_attention_append(cache, new_k, new_v, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx,
+                                    exact_q=True)
+    torch.cuda.synchronize()
+    assert cache.error_flags() == 0
+    err = helpers.max_abs_diff_groups(out.cpu().numpy(), wl, helpers.all_groups(wl), helpers.oracle_seq_exact_q)
+    assert err <= OUT_TOL, err
+
+
 # ------------------------------------------------------------------ decode
 
 def test_decode_parity_tiny(spkv):
