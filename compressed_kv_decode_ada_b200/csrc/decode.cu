@@ -646,8 +646,8 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
   // grid's CTAs leave, and each waits for the rows it merges
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   build_prefix(p.ctx_lens, p.B, p.Hkv, p.max_ctx, p.max_pages, p.err, P, scratch, tid, Ly::THREADS);
-  const int64_t W = P[p.B];
-  const int64_t u0 = split_begin(W, C, c), u1 = split_begin(W, C, c + 1);
+  const Partition part(P, p.B, p.Hkv, C);
+  const int64_t u0 = part.begin(c), u1 = part.begin(c + 1);
   if (u0 >= u1) return;  // uniform across the block
 
   if (tid == 0) {
@@ -1132,7 +1132,6 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint3
                                                     const int32_t *ctx_lens, int B, int Hkv, int Hq, int max_ctx,
                                                     int max_pages, void *out, int out_bf16, uint32_t *err) {
   constexpr int kChunk = 256;  // partials per pass
-  __shared__ int64_t red[2][4];
   __shared__ float wgt[kChunk];
   __shared__ float lsh[kChunk];
   __shared__ int64_t off[kChunk];
@@ -1141,35 +1140,19 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint3
   const int hq = blockIdx.x % Hq, b = blockIdx.x / Hq;
   const int h = hq / G, g = hq % G, bh = b * Hkv + h;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  int64_t before = 0, total = 0;
-  for (int i = tid; i < B; i += 128) {
-    const int np = seq_pages(ctx_lens[i], max_ctx, max_pages, nullptr) * Hkv;
-    total += np;
-    if (i < b) before += np;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    before += __shfl_xor_sync(0xffffffffu, before, o);
-    total += __shfl_xor_sync(0xffffffffu, total, o);
-  }
-  if (lane == 0) {
-    red[0][wid] = before;
-    red[1][wid] = total;
-  }
-  __syncthreads();
-  before = red[0][0] + red[0][1] + red[0][2] + red[0][3];
-  const int64_t W = red[1][0] + red[1][1] + red[1][2] + red[1][3];
-  const int np = seq_pages(ctx_lens[b], max_ctx, max_pages, nullptr);
+  __shared__ int32_t Psh[kMaxB + 1];
+  __shared__ int32_t pscr[8];
+  build_prefix(ctx_lens, B, Hkv, max_ctx, max_pages, nullptr, Psh, pscr, tid, 128);
+  const Partition part(Psh, B, Hkv, C);
+  const int np = (Psh[b + 1] - Psh[b]) / Hkv;
   float num = 0.f, den = 0.f;
   if (np > 0) {
-    const int64_t a = before + (int64_t)h * np, e = a + np;
-    const int64_t cf = ((a + 1) * C + W - 1) / W - 1;
-    int64_t cl = (e * C + W - 1) / W - 1;
-    if (cl > C - 1) cl = C - 1;
+    const int64_t a = (int64_t)Psh[b] + (int64_t)h * np, e = a + np;
+    const int64_t cf = part.split_of(a, bh), cl = part.split_of(e - 1, bh);
     // splits that hold units of the row (every split in [cf, cl] but empty ones)
     uint32_t live = 0;
     for (int64_t cc = cf + tid; cc <= cl; cc += 128)
-      live += split_begin(W, C, (int)cc) < split_begin(W, C, (int)cc + 1) ? 1u : 0u;
+      live += part.live_in_row(cc, cf, cl) ? 1u : 0u;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) live += __shfl_xor_sync(0xffffffffu, live, o);
     if (lane == 0) nred[wid] = live;
@@ -1197,7 +1180,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint3
       if (base + tid < nparts) {
         const int64_t cc = cf + (base + tid) / NCW;
         const int w = (int)((base + tid) % NCW);
-        if (split_begin(W, C, (int)cc) < split_begin(W, C, (int)cc + 1))
+        if (part.live_in_row(cc, cf, cl))
           mm = __ldcg(ws + (((cc + bh) * NCW + w) * G + g) * kPartial);
       }
       M = fmaxf(M, mm);
@@ -1215,7 +1198,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint3
           if (base + i < nparts) {
             const int64_t cc = cf + (base + i) / NCW;
             const int w = (int)((base + i) % NCW);
-            if (split_begin(W, C, (int)cc) < split_begin(W, C, (int)cc + 1)) {
+            if (part.live_in_row(cc, cf, cl)) {
               o = (((cc + bh) * NCW + w) * G + g) * kPartial;
               const float2 ml = __ldcg(reinterpret_cast<const float2 *>(ws + o));
               if (ml.x != kNegInf) {

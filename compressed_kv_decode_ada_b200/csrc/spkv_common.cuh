@@ -197,13 +197,64 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 // ------------------------------------------------------------ work partition
 // The (page, kv head) units of a batch are numbered u = P[b] + h * np_b + j
 // (sequence-major, then kv head, then page), where np_b = ceil(ctx_b / 16)
-// and P is the exclusive prefix sum of np_b * H_kv.  Split c of C owns the
-// contiguous units [floor(c W / C), floor((c+1) W / C)), W = P[B]; each
-// (split, kv-head row bh) intersection is a segment whose partial result goes
-// to workspace slot c + bh (unique because both indices only grow along the
-// unit order).
+// and P is the exclusive prefix sum of np_b * H_kv (W = P[B] units).  A kv row
+// r = b * H_kv + h holds units [rs(r), rs(r + 1)).  Split c of C owns a
+// contiguous range of units, cut at equal steps of a weighted position
+//   f(u) = u + kRowCostUnits * r(u),
+// i.e. every row boundary costs kRowCostUnits units: a split that crosses one
+// runs a second segment (query preparation, a warp barrier, partials) and gets
+// that many fewer pages.  With F = W + kRowCostUnits * B * H_kv and
+// t_c = floor(c F / C), split c begins at the first unit u with f(u) >= t_c.
+// Each (split, kv-head row bh) intersection is a segment whose partial result
+// goes to workspace slot c + bh (unique because both indices only grow along
+// the unit order).
+constexpr int64_t kRowCostUnits = 20;
 
-__device__ __forceinline__ int64_t split_begin(int64_t W, int C, int c) { return (W * (int64_t)c) / C; }
+struct Partition {
+  const int32_t *P;
+  int B, Hkv, C;
+  int64_t W, F;
+  __device__ __forceinline__ Partition(const int32_t *P_, int B_, int Hkv_, int C_)
+      : P(P_), B(B_), Hkv(Hkv_), C(C_) {
+    W = P[B];
+    F = W + kRowCostUnits * (int64_t)B * Hkv;
+  }
+  // weighted start of sequence b: f of its first unit (rows before it: b * Hkv)
+  __device__ __forceinline__ int64_t seq_f(int b) const { return (int64_t)P[b] + kRowCostUnits * (int64_t)b * Hkv; }
+  __device__ __forceinline__ int64_t target(int c) const { return (F * (int64_t)c) / C; }
+  // first unit of split c (begin(C) = W): the first u with f(u) >= t_c
+  __device__ __forceinline__ int64_t begin(int c) const {
+    if (c <= 0) return 0;
+    if (c >= C) return W;
+    const int64_t t = target(c);
+    int lo = 0, hi = B - 1;  // last sequence b with seq_f(b) <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (seq_f(mid) <= t) lo = mid;
+      else hi = mid - 1;
+    }
+    const uint32_t np = (uint32_t)(P[lo + 1] - P[lo]) / (uint32_t)Hkv;
+    const uint32_t d = (uint32_t)(t - seq_f(lo));  // < Hkv (np + k) + k, fits 32 bits
+    uint32_t h = d / (np + (uint32_t)kRowCostUnits);
+    if (h > (uint32_t)Hkv - 1u) h = (uint32_t)Hkv - 1u;
+    const int64_t rs = (int64_t)P[lo] + (int64_t)h * np;
+    const int64_t u = rs + (int64_t)(d - h * (np + (uint32_t)kRowCostUnits));
+    const int64_t re = rs + np;
+    return u < re ? u : re;  // t in the gap after the row: the next row's first unit
+  }
+  // the split whose units contain unit u of kv row r: the last c with t_c <= f(u)
+  __device__ __forceinline__ int64_t split_of(int64_t u, int64_t r) const {
+    const int64_t f = u + kRowCostUnits * r;
+    return ((f + 1) * C - 1) / F;
+  }
+  // For the splits [cf, cl] that meet one row (cf = split_of(first unit),
+  // cl = split_of(last unit)): cf and cl hold units of the row, and a split
+  // in between begins inside the row at a + t_c - f(a), so it holds units
+  // iff t_c < t_{c+1}.
+  __device__ __forceinline__ bool live_in_row(int64_t c, int64_t cf, int64_t cl) const {
+    return c == cf || c == cl || target((int)c) < target((int)c + 1);
+  }
+};
 
 // Pages of a sequence, validated against max_ctx and max_pages.
 __device__ __forceinline__ int seq_pages(int ctx, int max_ctx, int max_pages, uint32_t *err) {
