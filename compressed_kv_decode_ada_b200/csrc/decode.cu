@@ -139,12 +139,7 @@ struct Layout {
   static constexpr int QT_TIER = 2 * QT_HALF;
   static constexpr int QT_FLOATS = (ADA ? kTiers : 1) * QT_TIER;
   static constexpr int PBUF_FLOATS = NCW * G * 2 * kPage;      // p[g][32 slots of 2 pages] per warp
-  static constexpr int C2_BYTES = ADA ? 2 * kLutEntries * 8 : 0;   // fp64 edge tables (query coding)
   static constexpr int PB_BYTES = PBUF_FLOATS * 4;
-  // the edge tables are only read while the query is coded, the p buffers
-  // only while pages are processed: they share one region
-  static constexpr int PBC2_BYTES = PB_BYTES > C2_BYTES ? PB_BYTES : C2_BYTES;
-
   static constexpr int off_v = 0;                                 // NCW x 2 value slots
   static constexpr int off_x = off_v + NCW * 2 * VSLOT;           // ring stages
   // float2 single-angle tables: polar at off_lut, azimuth 384 entries later;
@@ -155,8 +150,8 @@ struct Layout {
   static constexpr int LAZ_OFF = 384;  // entries
   static constexpr int lut_bytes = ADA ? (LAZ_OFF + kLutEntries) * 8 : 0;
   static constexpr int off_qt = off_lut + lut_bytes;
-  static constexpr int off_pbc2 = off_qt + QT_FLOATS * 4;
-  static constexpr int off_sc = off_pbc2 + PBC2_BYTES;            // G scales + L_h + Delta_h
+  static constexpr int off_pbuf = off_qt + QT_FLOATS * 4;
+  static constexpr int off_sc = off_pbuf + PB_BYTES;            // G scales + L_h + Delta_h
   static constexpr int off_bar = off_sc + ((G + 2) * 4 + 15) / 16 * 16;  // full, empty, value slots
   static constexpr int off_meta = off_bar + (2 * NST + 2 * NCW) * 8;
   static constexpr int off_misc = off_meta + NST * 32;            // abort flag + scan scratch
@@ -624,12 +619,12 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
   float2 *lpol = reinterpret_cast<float2 *>(smem + Ly::off_lut);
   float2 *laz = lpol + Ly::LAZ_OFF;
   float *qt = reinterpret_cast<float *>(smem + Ly::off_qt);
-  double *pol_c2 = reinterpret_cast<double *>(smem + Ly::off_pbc2);
+  // fp64 edge tables of the exact code decisions (query coding, fused append),
+  // built once per CTA
+  double *pol_c2 = reinterpret_cast<double *>(smem + Ly::off_pe);
   double *az_c2 = pol_c2 + kLutEntries;
-  double *pe_pol = reinterpret_cast<double *>(smem + Ly::off_pe);  // producer's edge tables
-  double *pe_az = pe_pol + kLutEntries;
   uint8_t *pe_codes = smem + Ly::off_pe + 2 * kLutEntries * 8;
-  float *pbuf_all = reinterpret_cast<float *>(smem + Ly::off_pbc2);
+  float *pbuf_all = reinterpret_cast<float *>(smem + Ly::off_pbuf);
   float *sc = reinterpret_cast<float *>(smem + Ly::off_sc);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + Ly::off_bar);
   uint64_t *empty = full + NST;
@@ -656,10 +651,11 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
       mbar_init(&empty[s], 1);
     }
     for (int v = 0; v < NCW; ++v) mbar_init(&vbar_all[v], 1);
+    if (ADA) mbar_init(&vbar_all[NCW], 1);  // the consumers' tables are built (a spare slot)
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if constexpr (ADA) build_luts(lpol, laz, tid, Ly::THREADS);
+
   __syncthreads();
 
   const int n_units = (int)(u1 - u0);
@@ -708,7 +704,7 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
       }
       return r;
     };
-    bool pe_built = false;  // the producer's edge tables (built on the first append)
+    bool tables = false;
     A_ an = phaseA(0);
     B_ bn = phaseB(an);
     int k_last = -1;
@@ -748,17 +744,16 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
           // fused append: a row's last page gets the step's token before its copy
           uint32_t todo = p.new_k ? __ballot_sync(0xffffffffu, mine && valid && ac.last) : 0u;
           if (todo) {
-            if (!pe_built) {
-              build_edge_tables(pe_pol, pe_az, lane, 32);
-              __syncwarp();
-              pe_built = true;
+            if (!tables) {  // the fused append codes with the consumers' edge tables
+              mbar_wait_sleepy(&vbar_all[NCW], 0u, abort_flag, p.err);
+              tables = true;
             }
             while (todo) {
               const int src = __ffs(todo) - 1;
               todo &= todo - 1;
               append_token(p, __shfl_sync(0xffffffffu, ac.b, src), __shfl_sync(0xffffffffu, ac.h, src),
                            __shfl_sync(0xffffffffu, ac.pid, src), __shfl_sync(0xffffffffu, bc.bits, src),
-                           __shfl_sync(0xffffffffu, rec_off, src), pe_pol, pe_az, pe_codes, lane);
+                           __shfl_sync(0xffffffffu, rec_off, src), pol_c2, az_c2, pe_codes, lane);
             }
             // the copies below (and the consumers' value TMA) read what was written
             __threadfence();
@@ -816,6 +811,12 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
   uint64_t *const vbar = vbar_all + wid;  // the value pages of this warp's pair
   uint32_t vphase = 0u;
   int vpending = -1;  // phase of a value load a failed wait left in flight
+  if constexpr (ADA) {  // the consumers' tables, while the producer starts the ring
+    build_luts(lpol, laz, tid, NCW * 32);
+    build_edge_tables(pol_c2, az_c2, tid, NCW * 32);
+    named_bar_sync(1, NCW * 32);
+    if (tid == 0) mbar_arrive(&vbar_all[NCW]);
+  }
   int64_t u = u0;
   while (u < u1) {
     const int b = find_seq(P, p.B, u);
@@ -826,9 +827,7 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
     const int bh = b * p.Hkv + h;
 
     // ---- per-segment query preparation (every consumer warp is past the
-    // previous segment's last page: the edge tables may overwrite the p buffers)
-    named_bar_sync(1, NCW * 32);
-    if constexpr (ADA) build_edge_tables(pol_c2, az_c2, tid, NCW * 32);
+    // previous segment's last page: the query table may be rewritten)
     named_bar_sync(1, NCW * 32);
     for (int g = wid; g < G; g += NCW) {
       const uint16_t *qrow = p.q + ((int64_t)b * p.Hq + (int64_t)h * G + g) * kD;
