@@ -8,5 +8,5 @@ loudly when the CUDA library has not been built.
 from ._lib import LIB_PATH, SpkvError, lib  # noqa: F401
 from .cache import SpkvCache  # noqa: F401
 from .ops import (alloc_workspace, debug_logits, decode_attention, decode_attention_append,  # noqa: F401
-                  decode_attention_static_ws, decompress_then_dot, default_splits, dense_decode, encode_keys,
-                  workspace_bytes)
+                  decode_attention_partial, decode_attention_static_ws, decompress_then_dot, default_splits,
+                  dense_decode, encode_keys, merge_partials, workspace_bytes)

@@ -31,7 +31,10 @@ EXPORTS = (
     "spkv_decode_attention_ex",
     "spkv_debug_logits_ex",
     "spkv_decode_attention_append",
+    "spkv_decode_attention_partial",
+    "spkv_merge_partials",
 )
+PARTIAL_FLOATS = 132  # floats per (sequence, query head) shard record
 DECODE_EXACT_Q = 1  # SPKV_DECODE_EXACT_Q
 STATIC_WS_BYTES = 16 * 1024 * 1024  # SPKV_STATIC_WS_BYTES
 
@@ -100,6 +103,11 @@ def _load():
     L.spkv_decode_attention_append.restype = ctypes.c_int
     L.spkv_decode_attention_append.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _P, _P, _I, _I, _P, _I, _P, _I, _P,
                                                _I, _P, ctypes.c_size_t, _I, ctypes.c_uint32, _P]
+    L.spkv_decode_attention_partial.restype = ctypes.c_int
+    L.spkv_decode_attention_partial.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _I, _I, _P, _I, _P, _I, _P, _P,
+                                                ctypes.c_size_t, _I, ctypes.c_uint32, _P]
+    L.spkv_merge_partials.restype = ctypes.c_int
+    L.spkv_merge_partials.argtypes = [_P, _I, _I, _I, _P, _I, _P]
     L.spkv_debug_logits_ex.restype = ctypes.c_int
     L.spkv_debug_logits_ex.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _I, _I, _P, _I, _P, _I, _P, ctypes.c_uint32,
                                        _P]

@@ -1126,10 +1126,14 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
 // a block starts on an SM the split grid has left and waits (bounded) until
 // the row's count of written partials reaches NCW per covering split, so the
 // rows that finish early are merged while the last splits still run.
+// partial_out (optional): instead of out, the row's own partial record
+// (M, L, 0, 0, o[128]) with o = out, L = sum_s 2^(m_s - M) l_s, for a later
+// merge across shards of the sequences' pages (spkv_merge_partials).
 template <int G>
 __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint32_t *row_done, int C, int NCW,
                                                     const int32_t *ctx_lens, int B, int Hkv, int Hq, int max_ctx,
-                                                    int max_pages, void *out, int out_bf16, uint32_t *err) {
+                                                    int max_pages, void *out, int out_bf16, uint32_t *err,
+                                                    float *partial_out) {
   constexpr int kChunk = 256;  // partials per pass
   __shared__ float wgt[kChunk];
   __shared__ float lsh[kChunk];
@@ -1144,7 +1148,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint3
   build_prefix(ctx_lens, B, Hkv, max_ctx, max_pages, nullptr, Psh, pscr, tid, 128);
   const Partition part(Psh, B, Hkv, C);
   const int np = (Psh[b + 1] - Psh[b]) / Hkv;
-  float num = 0.f, den = 0.f;
+  float num = 0.f, den = 0.f, Mrow = kNegInf;
   if (np > 0) {
     const int64_t a = (int64_t)Psh[b] + (int64_t)h * np, e = a + np;
     const int64_t cf = part.split_of(a, bh), cl = part.split_of(e - 1, bh);
@@ -1189,6 +1193,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint3
     if (lane == 0) mred[wid] = M;
     __syncthreads();
     M = fmaxf(fmaxf(mred[0], mred[1]), fmaxf(mred[2], mred[3]));
+    Mrow = M;
     if (M != kNegInf) {
       for (int64_t base = 0; base < nparts; base += kChunk) {
         for (int i = tid; i < kChunk; i += 128) {
@@ -1226,7 +1231,39 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint3
     }
   }
   const float res = den > 0.f ? num / den : 0.f;
+  if (partial_out) {
+    float *pr = partial_out + ((int64_t)b * Hq + hq) * kPartial;
+    pr[4 + tid] = res;
+    if (tid == 0) *reinterpret_cast<float4 *>(pr) = make_float4(den > 0.f ? Mrow : kNegInf, den, 0.f, 0.f);
+    return;
+  }
   const int64_t o = ((int64_t)b * Hq + hq) * kD + tid;
+  if (out_bf16) reinterpret_cast<__nv_bfloat16 *>(out)[o] = __float2bfloat16_rn(res);
+  else reinterpret_cast<float *>(out)[o] = res;
+}
+
+// ------------------------------------------------------- shard merge kernel
+// One block per (sequence, query head): out = sum_r w_r o_r / sum_r w_r with
+// w_r = 2^(M_r - M) L_r over the R partial records (M_r = -inf: no weight);
+// 0 when no shard retained anything.
+__global__ void __launch_bounds__(128) merge_partials_kernel(const float *partials, int R, int BH, void *out,
+                                                             int out_bf16) {
+  const int row = blockIdx.x, tid = threadIdx.x;
+  float M = kNegInf;
+  for (int r = 0; r < R; ++r) M = fmaxf(M, partials[((int64_t)r * BH + row) * kPartial]);
+  float num = 0.f, den = 0.f;
+  if (M != kNegInf) {
+    for (int r = 0; r < R; ++r) {
+      const float *pr = partials + ((int64_t)r * BH + row) * kPartial;
+      const float2 ml = *reinterpret_cast<const float2 *>(pr);
+      if (ml.x == kNegInf) continue;
+      const float w = fast_exp2(ml.x - M) * ml.y;
+      num = fmaf(w, pr[4 + tid], num);
+      den += w;
+    }
+  }
+  const float res = den > 0.f ? num / den : 0.f;
+  const int64_t o = (int64_t)row * kD + tid;
   if (out_bf16) reinterpret_cast<__nv_bfloat16 *>(out)[o] = __float2bfloat16_rn(res);
   else reinterpret_cast<float *>(out)[o] = res;
 }
@@ -1411,6 +1448,7 @@ struct DecodeArgs {
   int G, num_splits;
   void *out;
   int out_bf16;
+  float *partial_out = nullptr;
 };
 
 template <bool ADA, int G, bool NW>
@@ -1436,7 +1474,8 @@ spkv_status launch_g(const DecodeArgs &a, const CUtensorMap &vmap, cudaStream_t 
   const float *ws = a.sp.ws;
   const uint32_t *done = a.sp.row_done;
   if (cudaLaunchKernelEx(&cfg, merge_kernel<G>, ws, done, a.num_splits, Ly::NCW, a.sp.ctx_lens, a.sp.B, a.sp.Hkv,
-                         a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16, a.sp.err) != cudaSuccess)
+                         a.sp.Hq, a.sp.max_ctx, a.sp.max_pages, a.out, a.out_bf16, a.sp.err,
+                         a.partial_out) != cudaSuccess)
     return SPKV_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
 }
@@ -1542,7 +1581,7 @@ namespace {
 spkv_status decode_ada(const spkv_cache *cache, const uint16_t *new_k, const uint16_t *new_v, const uint16_t *q,
                        int32_t B, int32_t Hq, const int32_t *block_table, int32_t max_pages, const int32_t *ctx_lens,
                        int32_t max_ctx, void *out, int32_t out_is_bf16, void *ws, size_t ws_bytes,
-                       int32_t num_splits, uint32_t flags, void *stream) {
+                       int32_t num_splits, uint32_t flags, void *stream, float *partial_out = nullptr) {
   if (flags & ~SPKV_DECODE_EXACT_Q) return SPKV_ERR_INVALID_ARG;
   spkv_status st = check_cache(cache);
   if (st != SPKV_OK) return st;
@@ -1557,10 +1596,32 @@ spkv_status decode_ada(const spkv_cache *cache, const uint16_t *new_k, const uin
   if (B == 0) return SPKV_OK;
   a.out = out;
   a.out_bf16 = out_is_bf16 ? 1 : 0;
+  a.partial_out = partial_out;
   return launch_split_and_merge<true>(a, (cudaStream_t)stream);
 }
 }  // namespace
 }  // namespace spkv
+
+extern "C" spkv_status spkv_decode_attention_partial(const spkv_cache *cache, const uint16_t *q, int32_t B,
+                                                     int32_t Hq, const int32_t *block_table, int32_t max_pages,
+                                                     const int32_t *ctx_lens, int32_t max_ctx, float *partial_out,
+                                                     void *ws, size_t ws_bytes, int32_t num_splits, uint32_t flags,
+                                                     void *stream) {
+  if (B > 0 && (!partial_out || ((uintptr_t)partial_out & 15))) return SPKV_ERR_INVALID_ARG;
+  // out is unused on this path; prep_batch only needs an aligned non-null pointer
+  return decode_ada(cache, nullptr, nullptr, q, B, Hq, block_table, max_pages, ctx_lens, max_ctx, partial_out, 0,
+                    ws, ws_bytes, num_splits, flags, stream, partial_out);
+}
+
+extern "C" spkv_status spkv_merge_partials(const float *partials, int32_t R, int32_t B, int32_t Hq, void *out,
+                                           int32_t out_is_bf16, void *stream) {
+  if (R < 1 || B < 0 || Hq < 1) return SPKV_ERR_INVALID_ARG;
+  if (B == 0) return SPKV_OK;
+  if (!partials || !out || ((uintptr_t)partials & 15) || ((uintptr_t)out & 15)) return SPKV_ERR_INVALID_ARG;
+  if ((int64_t)B * Hq > 0x7fffffff) return SPKV_ERR_UNSUPPORTED;
+  merge_partials_kernel<<<B * Hq, 128, 0, (cudaStream_t)stream>>>(partials, R, B * Hq, out, out_is_bf16 ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
+}
 
 extern "C" spkv_status spkv_decode_attention_ex(const spkv_cache *cache, const uint16_t *q, int32_t B, int32_t Hq,
                                                 const int32_t *block_table, int32_t max_pages,

@@ -10,7 +10,7 @@ import ctypes
 
 import torch
 
-from ._lib import DECODE_EXACT_Q, check, lib
+from ._lib import DECODE_EXACT_Q, PARTIAL_FLOATS, check, lib
 from .cache import HEAD_DIM, SpkvCache
 
 
@@ -136,6 +136,38 @@ def decode_attention_append(cache: SpkvCache, new_keys: torch.Tensor, new_values
                                            _ptr(out), int(out.dtype == torch.bfloat16), _ptr(ws), wsb,
                                            int(num_splits), DECODE_EXACT_Q if exact_q else 0, _stream(stream)),
           "spkv_decode_attention_append")
+    return out
+
+
+def decode_attention_partial(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tensor, ctx_lens: torch.Tensor,
+                             max_ctx: int, partial=None, ws=None, num_splits: int = 0, stream=None,
+                             exact_q: bool = False) -> torch.Tensor:
+    """spkv_decode_attention_partial: this shard's records [B, Hq, 132] (M, L, 0, 0, o[128])."""
+    _batch_checks(q, block_table, ctx_lens)
+    B, Hq, _ = q.shape
+    if partial is None:
+        partial = torch.empty((B, Hq, PARTIAL_FLOATS), dtype=torch.float32, device=q.device)
+    _need(partial, torch.float32, "partial", 3)
+    if tuple(partial.shape) != (B, Hq, PARTIAL_FLOATS):
+        raise ValueError("partial must be [B, Hq, 132]")
+    ws, wsb = _ws(ws, B, Hq, cache.num_kv_heads, max_ctx, num_splits, q.device)
+    c = cache.c_struct()
+    check(lib.spkv_decode_attention_partial(ctypes.byref(c), _ptr(q), B, Hq, _ptr(block_table), block_table.shape[1],
+                                            _ptr(ctx_lens), int(max_ctx), _ptr(partial), _ptr(ws), wsb,
+                                            int(num_splits), DECODE_EXACT_Q if exact_q else 0, _stream(stream)),
+          "spkv_decode_attention_partial")
+    return partial
+
+
+def merge_partials(partials: torch.Tensor, out=None, out_dtype=torch.float32, stream=None) -> torch.Tensor:
+    """spkv_merge_partials: combine shard records [R, B, Hq, 132] into out [B, Hq, 128]."""
+    _need(partials, torch.float32, "partials", 4)
+    R, B, Hq, n = partials.shape
+    if n != PARTIAL_FLOATS:
+        raise ValueError("partials must be [R, B, Hq, 132]")
+    out = _out_buffer(out, B, Hq, out_dtype, partials.device)
+    check(lib.spkv_merge_partials(_ptr(partials), R, B, Hq, _ptr(out), int(out.dtype == torch.bfloat16),
+                                  _stream(stream)), "spkv_merge_partials")
     return out
 
 

@@ -202,6 +202,31 @@ SPKV_API spkv_status spkv_decode_attention_append(const spkv_cache *cache, const
                                          int32_t out_is_bf16, void *ws, size_t ws_bytes, int32_t num_splits,
                                          uint32_t flags, void *stream);
 
+/* Page-sharded decode, for one long sequence (the 128K regime of the
+ * summary's section 4) whose pages are split across GPUs: each GPU decodes
+ * the pages it holds with this call and the shards are combined with
+ * spkv_merge_partials.  Same arguments and rules as spkv_decode_attention_ex
+ * (block_table / ctx_lens describe this shard's pages), but instead of the
+ * output it writes for every sequence b and query head hq the record
+ *   partial_out[b, hq, 0..131] = { M, L, 0, 0, o[0..127] }
+ *   M  max over the shard's retained tokens of logit * log2(e)  (-inf: none)
+ *   L  sum over them of 2^(logit * log2(e) - M)
+ *   o  the shard's own attention output (softmax over its tokens times V)
+ * partial_out: [B, Hq, 132] fp32, device, 16-byte aligned. */
+SPKV_API spkv_status spkv_decode_attention_partial(const spkv_cache *cache, const uint16_t *q, int32_t B,
+                                          int32_t num_q_heads, const int32_t *block_table, int32_t max_pages,
+                                          const int32_t *ctx_lens, int32_t max_ctx, float *partial_out, void *ws,
+                                          size_t ws_bytes, int32_t num_splits, uint32_t flags, void *stream);
+
+/* Combine R shard records of spkv_decode_attention_partial:
+ *   out[b, hq, :] = sum_r w_r o_r / sum_r w_r,  w_r = 2^(M_r - max_r M_r) L_r
+ * (shards with M_r = -inf carry no weight; 0 when no shard retained a token),
+ * which is the attention over the union of the shards' tokens.
+ *   partials [R, B, Hq, 132] fp32, device, 16-byte aligned (R >= 1)
+ *   out      [B, Hq, 128] fp32 or bf16 (out_is_bf16), device, 16-byte aligned */
+SPKV_API spkv_status spkv_merge_partials(const float *partials, int32_t R, int32_t B, int32_t num_q_heads,
+                                void *out, int32_t out_is_bf16, void *stream);
+
 /* Dense paged decode over bf16 keys, the uncompressed comparison path
  * (section 4 of the summary compares against dense KV):
  * logit = q . k / sqrt(128), same paging, mask, split and output rules as
