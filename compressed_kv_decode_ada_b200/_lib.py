@@ -33,6 +33,7 @@ EXPORTS = (
     "spkv_decode_attention_append",
     "spkv_decode_attention_partial",
     "spkv_merge_partials",
+    "spkv_debug_wait_timeout",
 )
 PARTIAL_FLOATS = 132  # floats per (sequence, query head) shard record
 DECODE_EXACT_Q = 1  # SPKV_DECODE_EXACT_Q
@@ -108,6 +109,8 @@ def _load():
                                                 ctypes.c_size_t, _I, ctypes.c_uint32, _P]
     L.spkv_merge_partials.restype = ctypes.c_int
     L.spkv_merge_partials.argtypes = [_P, _I, _I, _I, _P, _I, _P]
+    L.spkv_debug_wait_timeout.restype = ctypes.c_int
+    L.spkv_debug_wait_timeout.argtypes = [_P, _P, ctypes.c_uint64, _P]
     L.spkv_debug_logits_ex.restype = ctypes.c_int
     L.spkv_debug_logits_ex.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _I, _I, _P, _I, _P, _I, _P, ctypes.c_uint32,
                                        _P]

@@ -138,14 +138,15 @@ __device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity,
 // results of this call are flagged as invalid.
 // sleep_ns > 0 backs off between polls (for waiters off the critical path).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                                  uint32_t *err, uint32_t sleep_ns = 0) {
+                                                  uint32_t *err, uint32_t sleep_ns = 0,
+                                                  uint64_t limit_ns = 1000000000ull) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if ((it & 63u) == 63u && globaltimer_ns() - t0 > 1000000000ull) {
+    if ((it & 63u) == 63u && globaltimer_ns() - t0 > limit_ns) {
       *abort = 1;
       set_err(err, SPKV_DEVERR_TIMEOUT);
       return false;

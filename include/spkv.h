@@ -294,6 +294,17 @@ SPKV_API spkv_status spkv_debug_logits_ex(const spkv_cache *cache, const uint16_
                                  const int32_t *ctx_lens, int32_t max_ctx, float *logits, uint32_t flags,
                                  void *stream);
 
+/* Test hook for the bounded waits: one kernel waits, with the decode
+ * kernels' own bounded-wait routine, on an mbarrier that nothing completes,
+ * for at most limit_ns (1 .. 1e9 ns).  The wait gives up: it sets
+ * SPKV_DEVERR_TIMEOUT in *err_flags and the kernel returns normally, writing
+ *   status[0] = 1 (the wait gave up; 0 would mean it completed),
+ *   status[1] = microseconds waited, status[2] = 1 (the abort flag it raised).
+ * err_flags: one device word; status: 3 int32 on the device.  Invalid
+ * arguments: SPKV_ERR_INVALID_ARG, nothing launched.  (The pages have no
+ * counterpart: this checks the library's own failure handling.) */
+SPKV_API spkv_status spkv_debug_wait_timeout(uint32_t *err_flags, int32_t *status, uint64_t limit_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
