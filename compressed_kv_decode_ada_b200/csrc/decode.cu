@@ -1012,12 +1012,6 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
           xst[q] = xst_all + s * Ly::XSTAGE;
         }
       }
-      {  // the stages' previous phases were this warp's own: the test is exact
-        const int kn = 2 * (i + NCW);
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-          ready[q] = kn + q < ke && mbar_test_wait(&full[(kn + q) % NST], (uint32_t)((kn + q) / NST) & 1u);
-      }
       // the pair's value pages, into this warp's slots (overlaps the logits)
       const bool vload = use[0] || use[1];
       if (lane == 0 && vload) {
@@ -1055,6 +1049,14 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
         for (int q = 0; q < 2; ++q) {
           if (use[q]) page_logits(mt[q], xst[q], l2[q]);  // warp-uniform
         }
+      }
+      // test the next pair's stages now (their previous phases were this
+      // warp's own, so the test is exact); the answer is used after P.V
+      {
+        const int kn = 2 * (i + NCW);
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          ready[q] = kn + q < ke && mbar_test_wait(&full[(kn + q) % NST], (uint32_t)((kn + q) / NST) & 1u);
       }
       // the ring stages are free once the logits are known
       __syncwarp();
