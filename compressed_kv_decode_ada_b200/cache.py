@@ -64,7 +64,20 @@ class SpkvCache:
             self.keep_mask = torch.from_numpy(km.view(np.int16)).to(self.device)
         self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
 
+    _DESCRIBED = frozenset(("num_pages", "num_kv_heads", "arena", "arena_bytes", "hdr", "v_pages", "rad_lo",
+                            "rad_step", "keep_mask", "err", "tiers"))
+
+    def __setattr__(self, name, value):
+        if name in self._DESCRIBED:  # the cached descriptor no longer matches
+            object.__setattr__(self, "_c", None)
+        object.__setattr__(self, name, value)
+
     def c_struct(self) -> SpkvCacheC:
+        """The spkv_cache descriptor of these buffers (rebuilt only after one
+        of them is replaced)."""
+        c = getattr(self, "_c", None)
+        if c is not None:
+            return c
         c = SpkvCacheC()
         c.num_kv_heads = self.num_kv_heads
         c.head_dim = HEAD_DIM
@@ -79,6 +92,7 @@ class SpkvCache:
         c.keep_mask = self.keep_mask.data_ptr() if self.keep_mask is not None else None
         c.err_flags = self.err.data_ptr()
         c.tiers = self.tiers
+        self._c = c
         return c
 
     def error_flags(self) -> int:

@@ -88,8 +88,9 @@ def _batch_checks(q, block_table, ctx_lens):
 
 
 def _ws(ws, B, Hq, Hkv, max_ctx, num_splits, device):
-    need = workspace_bytes(B, Hq, Hkv, max_ctx, num_splits)
+    # a caller's workspace is passed as is: the library checks its size
     if ws is None:
+        need = workspace_bytes(B, Hq, Hkv, max_ctx, num_splits)
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
     return ws, ws.numel() * ws.element_size()
 
