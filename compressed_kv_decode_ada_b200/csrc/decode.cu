@@ -536,6 +536,83 @@ __device__ __forceinline__ void ada_2page_f4(const uint8_t *recA, const uint8_t 
   }
 }
 
+// Pair path for any width b (used for b = 3, 6, 8; b = 4 has ada_2page_f4):
+// a rolled loop of two iterations, each decoding 32 fields of both pages --
+// 32 b bits = b whole words of the slot's stream, loaded per iteration -- so
+// the loop body stays one granule long whatever b is.
+template <int BITS, int G, int QT_HALF>
+__device__ __forceinline__ void ada_2page_gen(const uint8_t *recA, const uint8_t *recB, const float *qt,
+                                              const float2 *lpol, const float2 *laz, int lane, float (&fA)[G],
+                                              float (&fB)[G]) {
+  const int t = lane & 15, half = lane >> 4;
+  const float *qh = qt + half * QT_HALF;
+  const uint32_t *ra32 = reinterpret_cast<const uint32_t *>(recA);
+  const uint32_t *rb32 = reinterpret_cast<const uint32_t *>(recB);
+  float2 acc[2][G];
+  float Ps[2] = {1.f, 1.f};
+#pragma unroll
+  for (int pg = 0; pg < 2; ++pg)
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[pg][g] = make_float2(0.f, 0.f);
+#pragma unroll 1
+  for (int it = 0; it < 2; ++it) {
+    const int w0 = (2 * half + it) * BITS;  // first stream word of fields 64 half + 32 it ..
+    uint32_t WA[BITS], WB[BITS];
+#pragma unroll
+    for (int j = 0; j < BITS; ++j) {  // word w of the stream: chunk w / 4, word w % 4 of the slot's 16 bytes
+      const int w = w0 + j;
+      WA[j] = ra32[(16 * (w >> 2) + t) * 4 + (w & 3)];
+      WB[j] = rb32[(16 * (w >> 2) + t) * 4 + (w & 3)];
+    }
+    const bool tail = it == 1 && half;  // the granule's last pair is (azimuth, padding)
+    const float *qi = qh + it * 16 * G * 2;
+#pragma unroll
+    for (int pq = 0; pq < 16; ++pq) {
+      float2 uu[2];
+#pragma unroll
+      for (int pg = 0; pg < 2; ++pg) {
+        const uint32_t c0 = bits_at<BITS, BITS>(pg ? WB : WA, 2 * pq * BITS);
+        const uint32_t c1 = bits_at<BITS, BITS>(pg ? WB : WA, (2 * pq + 1) * BITS);
+        float2 e0, e1;
+        if (pq == 15) {
+          e0 = (tail ? laz : lpol)[c0];
+          const float2 t1 = lpol[c1];
+          e1 = make_float2(tail ? 1.0f : t1.x, tail ? 0.0f : t1.y);
+        } else {
+          e0 = lpol[c0];
+          e1 = lpol[c1];
+        }
+        const float u0 = Ps[pg] * e0.x, tt = Ps[pg] * e0.y;
+        uu[pg] = make_float2(u0, tt * e1.x);
+        Ps[pg] = tt * e1.y;
+      }
+      const float *qp = qi + pq * G * 2;
+      if constexpr (G == 1) {
+        const float2 q2 = *reinterpret_cast<const float2 *>(qp);
+        acc[0][0] = ffma2(uu[0], q2, acc[0][0]);
+        acc[1][0] = ffma2(uu[1], q2, acc[1][0]);
+      } else {
+#pragma unroll
+        for (int g = 0; g < G; g += 2) {
+          const float4 q4 = *reinterpret_cast<const float4 *>(qp + 2 * g);
+          const float2 qa = make_float2(q4.x, q4.y), qb = make_float2(q4.z, q4.w);
+          acc[0][g] = ffma2(uu[0], qa, acc[0][g]);
+          acc[0][g + 1] = ffma2(uu[0], qb, acc[0][g + 1]);
+          acc[1][g] = ffma2(uu[1], qa, acc[1][g]);
+          acc[1][g + 1] = ffma2(uu[1], qb, acc[1][g + 1]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float Aa = acc[0][g].x + acc[0][g].y, Ab = acc[1][g].x + acc[1][g].y;
+    const float Ba = __shfl_down_sync(0xffffffffu, Aa, 16), Bb = __shfl_down_sync(0xffffffffu, Ab, 16);
+    fA[g] = fmaf(Ps[0], Ba, Aa);
+    fB[g] = fmaf(Ps[1], Bb, Ab);
+  }
+}
+
 // --------------------------------------------------------- dense pieces
 // q (scaled by log2(e)/sqrt(d)) as fp32 in [half][chunk][g][8] with a 16-byte
 // skew per chunk so that lanes reading rotated chunks hit distinct banks.
@@ -673,10 +750,11 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
       int bits;
       uint32_t keep;
     };
-    auto phaseA = [&](int kb) -> A_ {
+    // units [u0 + kb + lane] below CTA-relative unit `lim`
+    auto phaseA = [&](int kb, int lim) -> A_ {
       A_ a{0, 0, 0, 0, 0, 0};
       const int k = kb + lane;
-      if (k < n_units) {
+      if (k < lim) {
         const int64_t u = u0 + k;
         const int b = find_seq(P, p.B, u);
         const int np = (P[b + 1] - P[b]) / p.Hkv;
@@ -704,16 +782,14 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
       }
       return r;
     };
-    bool tables = false;
-    A_ an = phaseA(0);
-    B_ bn = phaseB(an);
-    int k_last = -1;
-    for (int kb = 0; kb < n_units; kb += 32) {
-      const A_ ac = an;
-      const B_ bc = bn;
-      int valid = 0;
-      uint64_t rec_off = 0, v_off = 0;
-      uint32_t rec_sz = 0;
+    // a unit's copy plan: checks (flagging bad pages), record and value offsets
+    struct U_ {
+      int valid;
+      uint64_t rec_off, v_off;
+      uint32_t rec_sz, live;
+    };
+    auto plan = [&](const A_ &ac, const B_ &bc) -> U_ {
+      U_ x{0, 0, 0, 0, 0};
       if (ac.ok) {
         const int ti = tier_of_bits(bc.bits);
         if (ac.pid < 0 || ac.pid >= p.num_pages) {
@@ -721,72 +797,190 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
         } else if (ADA && (ti < 0 || !((p.tiers >> ti) & 1u))) {
           set_err(p.err, SPKV_DEVERR_BITS);
         } else {
-          v_off = ((uint64_t)ac.pid * p.Hkv + ac.h) * (kPage * kD);
+          x.v_off = ((uint64_t)ac.pid * p.Hkv + ac.h) * (kPage * kD);
           if constexpr (ADA) {
-            rec_sz = rec_bytes(bc.bits);
-            rec_off = (uint64_t)bc.off16 * 16u + (uint64_t)ac.h * rec_sz;
-            if (rec_off + rec_sz > p.arena_bytes) set_err(p.err, SPKV_DEVERR_RECORD);
-            else valid = 1;
+            x.rec_sz = rec_bytes(bc.bits);
+            x.rec_off = (uint64_t)bc.off16 * 16u + (uint64_t)ac.h * x.rec_sz;
+            if (x.rec_off + x.rec_sz > p.arena_bytes) set_err(p.err, SPKV_DEVERR_RECORD);
+            else x.valid = 1;
           } else {
-            valid = 1;
+            x.valid = 1;
           }
         }
       }
-      const uint32_t live = bc.keep & ((1u << ac.ntok) - 1u);
-      an = phaseA(kb + 32);
-      const int cnt = min(32, n_units - kb);
-      // lanes [i0, i0 + kIssue) wait for their own stages and issue together
-      for (int i0 = 0; i0 < cnt; i0 += kIssue) {
-        if (i0 == 16) bn = phaseB(an);
-        const int k = kb + lane, s = k % NST, r = k / NST;
-        const bool mine = lane >= i0 && lane < i0 + kIssue && lane < cnt;
-        if constexpr (ADA) {
-          // fused append: a row's last page gets the step's token before its copy
-          uint32_t todo = p.new_k ? __ballot_sync(0xffffffffu, mine && valid && ac.last) : 0u;
-          if (todo) {
-            if (!tables) {  // the fused append codes with the consumers' edge tables
-              mbar_wait_sleepy(&vbar_all[NCW], 0u, abort_flag, p.err);
-              tables = true;
-            }
-            while (todo) {
-              const int src = __ffs(todo) - 1;
-              todo &= todo - 1;
-              append_token(p, __shfl_sync(0xffffffffu, ac.b, src), __shfl_sync(0xffffffffu, ac.h, src),
-                           __shfl_sync(0xffffffffu, ac.pid, src), __shfl_sync(0xffffffffu, bc.bits, src),
-                           __shfl_sync(0xffffffffu, rec_off, src), pol_c2, az_c2, pe_codes, lane);
-            }
-            // the copies below (and the consumers' value TMA) read what was written
-            __threadfence();
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            __syncwarp();
+      x.live = bc.keep & ((1u << ac.ntok) - 1u);
+      return x;
+    };
+    bool tables = false;
+    // One issue step (warp-wide): the lanes with `mine` set fill their units'
+    // stages s = k % NST (at most kIssue distinct stages per step).
+    auto issue = [&](const A_ &ac, const B_ &bc, const U_ &x, bool mine, int k) {
+      const int s = k % NST, r = k / NST;
+      if constexpr (ADA) {
+        // fused append: a row's last page gets the step's token before its copy
+        uint32_t todo = p.new_k ? __ballot_sync(0xffffffffu, mine && x.valid && ac.last) : 0u;
+        if (todo) {
+          if (!tables) {  // the fused append codes with the consumers' edge tables
+            mbar_wait_sleepy(&vbar_all[NCW], 0u, abort_flag, p.err);
+            tables = true;
+          }
+          while (todo) {
+            const int src = __ffs(todo) - 1;
+            todo &= todo - 1;
+            append_token(p, __shfl_sync(0xffffffffu, ac.b, src), __shfl_sync(0xffffffffu, ac.h, src),
+                         __shfl_sync(0xffffffffu, ac.pid, src), __shfl_sync(0xffffffffu, bc.bits, src),
+                         __shfl_sync(0xffffffffu, x.rec_off, src), pol_c2, az_c2, pe_codes, lane);
+          }
+          // the copies below (and the consumers' value TMA) read what was written
+          __threadfence();
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          __syncwarp();
+        }
+      }
+      if (mine) {
+        if (r > 0) mbar_wait_sleepy(&empty[s], (uint32_t)(r - 1) & 1u, abort_flag, p.err);
+        StageMeta m;
+        m.valid = x.valid && !*abort_flag;
+        m.bits = bc.bits;
+        m.ntok = ac.ntok;
+        m.live = x.live;
+        m.vrow = (int)(x.v_off / kD);  // (pid * H_kv + h) * 16
+        meta[s] = m;
+        uint8_t *xst = xst_all + s * Ly::XSTAGE;
+        if (m.valid) {
+          if constexpr (ADA) {
+            mbar_arrive_expect_tx(&full[s], x.rec_sz);
+            bulk_g2s(xst, p.arena + x.rec_off, x.rec_sz, &full[s]);
+          } else {
+            mbar_arrive_expect_tx(&full[s], 4096u);
+            bulk_g2s(xst, p.k_pages + x.v_off, 4096u, &full[s]);
+          }
+        } else {
+          mbar_arrive(&full[s]);
+        }
+      }
+      __syncwarp();
+    };
+    int k_last = -1;
+    if (ADA && !NW && __popc(p.tiers) > 1) {
+      // Several tiers (wide caches; a narrow cache's b = 3 and b = 4 both pair): a kv row's pages may be decoded in any order (softmax
+      // and P.V run over the set), so each segment is walked once per tier
+      // present and that tier's pages take the next units.  Long runs of one
+      // tier keep neighbouring units paired and every warp on one code path.
+      // (Pages whose header names no tier of the mask go with the first pass,
+      // as units the consumers skip.)
+      const int t_first = __ffs(p.tiers) - 1;
+      int next_k = 0;
+      int sa = 0;
+      while (sa < n_units) {
+        const int64_t ua = u0 + sa;
+        const int b = find_seq(P, p.B, ua);
+        const int np = (P[b + 1] - P[b]) / p.Hkv;
+        const int h = (int)((ua - P[b]) / np);
+        const int64_t seg_hi = (int64_t)P[b] + (int64_t)(h + 1) * np;
+        const int se = (int)((seg_hi < u1 ? seg_hi : u1) - u0);
+        for (int t = t_first; t < kTiers; ++t) {
+          if (!((p.tiers >> t) & 1u)) continue;
+          for (int sb = sa; sb < se; sb += 32) {
+            const A_ ac = phaseA(sb, se);
+            const B_ bc = phaseB(ac);
+            const U_ x = plan(ac, bc);
+            const int ti = tier_of_bits(bc.bits);
+            const bool in_mask = ti >= 0 && ((p.tiers >> ti) & 1u);
+            const bool sel = ac.ok && (in_mask ? ti == t : t == t_first);
+            const uint32_t sm = __ballot_sync(0xffffffffu, sel);
+            const int rank = __popc(sm & ((1u << lane) - 1u)), nsel = __popc(sm);
+            for (int i0 = 0; i0 < nsel; i0 += kIssue)
+              issue(ac, bc, x, sel && rank >= i0 && rank < i0 + kIssue, next_k + rank);
+            next_k += nsel;
           }
         }
-        if (mine) {
-          if (r > 0) mbar_wait_sleepy(&empty[s], (uint32_t)(r - 1) & 1u, abort_flag, p.err);
-          StageMeta m;
-          m.valid = valid && !*abort_flag;
-          m.bits = bc.bits;
-          m.ntok = ac.ntok;
-          m.live = live;
-          m.vrow = (int)(v_off / kD);  // (pid * H_kv + h) * 16
-          meta[s] = m;
-          uint8_t *xst = xst_all + s * Ly::XSTAGE;
-          if (m.valid) {
+        sa = se;
+      }
+      k_last = next_k - 1;
+    } else {
+      A_ an = phaseA(0, n_units);
+      B_ bn = phaseB(an);
+      for (int kb = 0; kb < n_units; kb += 32) {
+        const A_ ac = an;
+        const B_ bc = bn;
+        int valid = 0;
+        uint64_t rec_off = 0, v_off = 0;
+        uint32_t rec_sz = 0;
+        if (ac.ok) {
+          const int ti = tier_of_bits(bc.bits);
+          if (ac.pid < 0 || ac.pid >= p.num_pages) {
+            set_err(p.err, SPKV_DEVERR_PAGE_ID);
+          } else if (ADA && (ti < 0 || !((p.tiers >> ti) & 1u))) {
+            set_err(p.err, SPKV_DEVERR_BITS);
+          } else {
+            v_off = ((uint64_t)ac.pid * p.Hkv + ac.h) * (kPage * kD);
             if constexpr (ADA) {
-              mbar_arrive_expect_tx(&full[s], rec_sz);
-              bulk_g2s(xst, p.arena + rec_off, rec_sz, &full[s]);
+              rec_sz = rec_bytes(bc.bits);
+              rec_off = (uint64_t)bc.off16 * 16u + (uint64_t)ac.h * rec_sz;
+              if (rec_off + rec_sz > p.arena_bytes) set_err(p.err, SPKV_DEVERR_RECORD);
+              else valid = 1;
             } else {
-              mbar_arrive_expect_tx(&full[s], 4096u);
-              bulk_g2s(xst, p.k_pages + v_off, 4096u, &full[s]);
+              valid = 1;
             }
-          } else {
-            mbar_arrive(&full[s]);
           }
         }
-        __syncwarp();
+        const uint32_t live = bc.keep & ((1u << ac.ntok) - 1u);
+        an = phaseA(kb + 32, n_units);
+        const int cnt = min(32, n_units - kb);
+        // lanes [i0, i0 + kIssue) wait for their own stages and issue together
+        for (int i0 = 0; i0 < cnt; i0 += kIssue) {
+          if (i0 == 16) bn = phaseB(an);
+          const int k = kb + lane, s = k % NST, r = k / NST;
+          const bool mine = lane >= i0 && lane < i0 + kIssue && lane < cnt;
+          if constexpr (ADA) {
+            // fused append: a row's last page gets the step's token before its copy
+            uint32_t todo = p.new_k ? __ballot_sync(0xffffffffu, mine && valid && ac.last) : 0u;
+            if (todo) {
+              if (!tables) {  // the fused append codes with the consumers' edge tables
+                mbar_wait_sleepy(&vbar_all[NCW], 0u, abort_flag, p.err);
+                tables = true;
+              }
+              while (todo) {
+                const int src = __ffs(todo) - 1;
+                todo &= todo - 1;
+                append_token(p, __shfl_sync(0xffffffffu, ac.b, src), __shfl_sync(0xffffffffu, ac.h, src),
+                             __shfl_sync(0xffffffffu, ac.pid, src), __shfl_sync(0xffffffffu, bc.bits, src),
+                             __shfl_sync(0xffffffffu, rec_off, src), pol_c2, az_c2, pe_codes, lane);
+              }
+              // the copies below (and the consumers' value TMA) read what was written
+              __threadfence();
+              asm volatile("fence.proxy.async.global;" ::: "memory");
+              __syncwarp();
+            }
+          }
+          if (mine) {
+            if (r > 0) mbar_wait_sleepy(&empty[s], (uint32_t)(r - 1) & 1u, abort_flag, p.err);
+            StageMeta m;
+            m.valid = valid && !*abort_flag;
+            m.bits = bc.bits;
+            m.ntok = ac.ntok;
+            m.live = live;
+            m.vrow = (int)(v_off / kD);  // (pid * H_kv + h) * 16
+            meta[s] = m;
+            uint8_t *xst = xst_all + s * Ly::XSTAGE;
+            if (m.valid) {
+              if constexpr (ADA) {
+                mbar_arrive_expect_tx(&full[s], rec_sz);
+                bulk_g2s(xst, p.arena + rec_off, rec_sz, &full[s]);
+              } else {
+                mbar_arrive_expect_tx(&full[s], 4096u);
+                bulk_g2s(xst, p.k_pages + v_off, 4096u, &full[s]);
+              }
+            } else {
+              mbar_arrive(&full[s]);
+            }
+          }
+          __syncwarp();
+        }
+        k_last = kb + cnt - 1;
+        if (cnt <= 16) bn = phaseB(an);
       }
-      k_last = kb + cnt - 1;
-      if (cnt <= 16) bn = phaseB(an);
     }
     // On an abort, copies may still be in flight into our stages: wait for
     // them (bounded) before the CTA's shared memory can be released.
@@ -1023,7 +1217,7 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
       float l2[2][G];
       bool paired = false;
       if constexpr (ADA) {
-        paired = use[0] && use[1] && mt[0].bits == mt[1].bits && mt[0].bits <= 4;
+        paired = use[0] && use[1] && mt[0].bits == mt[1].bits && (!NW || mt[0].bits <= 4);
       }
       if (paired) {
         if constexpr (ADA) {
@@ -1031,10 +1225,19 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
           const int ti = tier_of_bits(mt[0].bits);
           const float *q0 = qt + ti * Ly::QT_TIER;
           const float2 *lp = lpol + lut_off(ti), *la = laz + lut_off(ti);
-          if (mt[0].bits == 4)
-            ada_2page_f4<G, Ly::QT_HALF>(xst[0], xst[1], q0, smem_u32(lp), smem_u32(la), lane, fa, fb);
-          else
-            ada_2page_f<3, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb);
+          if constexpr (NW) {
+            if (mt[0].bits == 4)
+              ada_2page_f4<G, Ly::QT_HALF>(xst[0], xst[1], q0, smem_u32(lp), smem_u32(la), lane, fa, fb);
+            else
+              ada_2page_f<3, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb);
+          } else {
+            switch (mt[0].bits) {
+              case 4: ada_2page_f4<G, Ly::QT_HALF>(xst[0], xst[1], q0, smem_u32(lp), smem_u32(la), lane, fa, fb); break;
+              case 3: ada_2page_gen<3, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb); break;
+              case 6: ada_2page_gen<6, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb); break;
+              default: ada_2page_gen<8, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb); break;
+            }
+          }
           const int bits = mt[0].bits;
           const float ra = fast_exp2(fmaf((float)xst[0][256 * bits + (lane & 15)], Dh, Lh));
           const float rb = fast_exp2(fmaf((float)xst[1][256 * bits + (lane & 15)], Dh, Lh));
