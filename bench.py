@@ -346,6 +346,19 @@ def compare_paths(args, spkv, workload, wl, cache, ctx, max_ctx, splits, ws, str
     return res
 
 
+def decode_code_hash() -> str:
+    """sha256[:16] of csrc/decode.cu with comments and blank lines removed:
+    the key under which a DRAM-traffic capture stays valid (a comment edit
+    does not change the kernel it describes)."""
+    import re
+
+    src = open(os.path.join(ROOT, "compressed_kv_decode_ada_b200", "csrc", "decode.cu")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
 def _committed_traffic(workload):
     """ncu DRAM bytes per launch of the ADA split kernel, from the committed
     profile summary, if it was taken on the current kernel source."""
@@ -355,10 +368,8 @@ def _committed_traffic(workload):
             d = json.load(f)
     except Exception:
         return None
-    src = os.path.join(ROOT, "compressed_kv_decode_ada_b200", "csrc", "decode.cu")
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     ent = d.get(workload)
-    if not ent or ent.get("decode_cu_sha256_16") != sha:
+    if not ent or ent.get("decode_cu_code_sha256_16") != decode_code_hash():
         return None
     return ent.get("dram_bytes_per_launch")
 

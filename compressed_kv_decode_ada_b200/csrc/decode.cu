@@ -14,24 +14,30 @@
 //
 // Kernel design (B200):
 //  * Work = (page, kv head) units of the whole ragged batch, numbered
-//    sequence-major; split c of C owns a contiguous, equal share (balanced for
-//    any mix of context lengths), so C = SMs x resident CTAs is one full wave.
-//  * CTA = 1 producer warp + 4 consumer warps.  The producer resolves block
-//    table -> page header -> record address and streams each unit's code
-//    record (256 b + 16 bytes) and its 4 KB value page into a shared-memory
-//    ring with 1-D bulk copies (cp.async.bulk, mbarrier completion).  Consumer
-//    warp w takes units w, w+4, ... and keeps its own online-softmax state.
-//  * f_b: lane = (slot t, half of the angle chain).  Each lane decodes 64
-//    angle codes of its slot, looks up (cos, sin) of the cell midpoint in a
-//    shared-memory table and runs the prefix product of sines
+//    sequence-major; split c of C owns a contiguous range cut at equal steps
+//    of a weighted position (every kv-row boundary costs a few units: see
+//    Partition), so C = 2 x SMs CTAs is one balanced wave.
+//  * CTA = 1 producer warp + 5 consumer warps (4 for G = 8), 2 CTAs per SM.
+//    The producer resolves block table -> page header -> record address and
+//    streams each unit's code record (256 b + 16 bytes) into a shared-memory
+//    ring with 1-D bulk copies (cp.async.bulk, mbarrier completion); with
+//    several tiers it walks each segment tier by tier.  Consumer warp w takes
+//    pairs of units w, w + NCW, ..., fetches the pair's value pages itself
+//    (3-D TMA, 128-byte swizzle) and keeps its own online-softmax state.
+//  * f_b: lane = (slot t, half of the angle chain) of both pages of a pair.
+//    Each lane decodes 64 angle codes per page, looks up (cos, sin) of the
+//    cell midpoint in a shared-memory table and runs the prefix product of
+//    sines
 //        u_j = (prod_{i<j} sin phi_i) cos phi_j,
 //    accumulating <u_q, u_k> for the G query heads of the kv head on CUDA
 //    cores (f32x2 FMAs).  The two halves are joined by
 //        f = A + (prod_{i<=64} sin phi_i) * B.
 //    The key's unit vector lives only in registers.
-//  * Online softmax in the log2 domain; P.V with lane = 4 value dims.
-//  * Per segment the 4 warps' states are merged and written as one partial
-//    (m, l, acc[128]) per query head; a second kernel merges the partials.
+//  * Online softmax in the log2 domain with a lazily moving maximum; P.V on
+//    tensor cores (mma.sync m16n8k16 bf16, P split into bf16 hi + lo).
+//  * Per segment every consumer warp writes one partial (m, l, acc[128]) per
+//    query head and counts it on its kv row; the merge kernel, launched as a
+//    programmatic dependent, merges each row once its partials are counted.
 #include <cuda_bf16.h>
 
 #include <type_traits>
@@ -112,8 +118,8 @@ __device__ __forceinline__ float warp_max(float x) {
 // ----------------------------------------------------------------- layout
 template <bool ADA, int G, bool NW = false>
 struct Layout {
-  // 5 consumer warps take PAIRS of units (ADA: the two pages of a pair that
-  // share a tier b <= 4 share every query load).  The producer warp streams
+  // NCW consumer warps take PAIRS of units (ADA: the two pages of a pair that
+  // share a tier share every query load).  The producer warp streams
   // only the small per-unit data -- the code record (ADA) or the bf16 K page
   // (dense) -- through a CTA-wide ring of NST stages; each consumer warp
   // fetches the value pages of its pair itself, into two private slots, when
@@ -129,10 +135,10 @@ struct Layout {
   // with NST / 2 a multiple of NCW every use of a stage is by one warp, in
   // order: its parity waits always target the current or the next phase.
   static_assert((NST / 2) % NCW == 0, "a stage must belong to one consumer warp");
-  // Value pages land through two 2-D TMA boxes (16 rows x 64 bf16, 128-byte
-  // swizzle): box j holds dims 64 j .. 64 j + 63, row t's 16-byte chunk c
-  // sits at chunk c ^ (t & 7), so the transposing ldmatrix reads of 8
-  // consecutive rows hit 8 distinct bank groups.  1024-byte aligned.
+  // A value page lands through one 3-D TMA box (64 dims x 16 rows x 2 halves,
+  // 128-byte swizzle): half j (dims 64 j .. 64 j + 63) at +2048 j, row t's
+  // 16-byte chunk c at chunk c ^ (t & 7), so the transposing ldmatrix reads
+  // of 8 consecutive rows hit 8 distinct bank groups.  1024-byte aligned.
   static constexpr int VSLOT = 4096;
   static constexpr int XSTAGE = ADA ? (NW ? 1040 : 2064) : 4096;  // code record | dense K page
   static constexpr int QT_HALF = ADA ? (64 * G + 4) : 8 * (8 * G + 4);  // floats, +16 B skew
