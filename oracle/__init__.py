@@ -76,6 +76,8 @@ def lib():
         L.spkv_oracle_decompress.argtypes = [_i, _i, _p, _p, _p, _d, _d, _p]
         L.spkv_oracle_ada_group.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _d, _d, _p, _p, _p, _p]
         L.spkv_oracle_ada_group_exact_q.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _d, _d, _p, _p, _p, _p]
+        L.spkv_oracle_rdr_plan.restype = _i
+        L.spkv_oracle_rdr_plan.argtypes = [_i, _i, _i, _p, _p, _p, _d, ctypes.c_uint32, _p, _p, _p, _p]
         L.spkv_oracle_dense_group.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _p]
         _lib = L
     return _lib
@@ -250,3 +252,18 @@ def map_groups(fn, items, threads: int | None = None):
     threads = threads or len(os.sched_getaffinity(0))
     with ThreadPoolExecutor(max_workers=threads) as ex:
         return list(ex.map(fn, items))
+
+
+def rdr_plan(keys_bf16, q_norms, budget_bytes, tier_mask=0xF, protect=None):
+    """RDR controller (readings R14-R17): tiers [T] (0 = evicted) for keys [T, H_kv, d].
+
+    Returns (tiers, lambda, rate_bytes, distortion, status)."""
+    k = _c(keys_bf16, np.uint16)
+    T, Hkv, d = k.shape
+    qn = _c(np.asarray(q_norms, np.float64).reshape(Hkv), np.float64)
+    pr = _c(protect, np.uint8)
+    tiers = np.empty(T, np.int32)
+    lam, rate, dist = (ctypes.c_double() for _ in range(3))
+    st = lib().spkv_oracle_rdr_plan(d, T, Hkv, _ptr(k), _ptr(qn), _ptr(pr), float(budget_bytes), int(tier_mask),
+                                    _ptr(tiers), ctypes.byref(lam), ctypes.byref(rate), ctypes.byref(dist))
+    return tiers, lam.value, rate.value, dist.value, int(st)

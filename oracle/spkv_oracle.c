@@ -364,3 +364,105 @@ void spkv_oracle_dense_group(int d, int G, int T, const uint16_t *q, const uint1
     }
     free(lg); free(kp);
 }
+
+/* ------------------------------------------------------------ RDR controller
+ * Rate-distortion retention (technical summary section 2.2): for every
+ * state, a residency decision and a precision tier under a hard memory
+ * budget, from a distortion surrogate built on the angular error of the
+ * codes scaled by the query and key magnitudes, with protected states kept
+ * at the top tier.  The section leaves the formulas open; the readings are:
+ *   R14 the decision unit is a token: its kv heads share a page, so they
+ *       share its tier b (b = 0: evicted);
+ *   R15 distortion D_t(b) = w_t eps_b with w_t = sum_h qn_h ||k_{t,h}|| and
+ *       eps_b = pi / (2^b sqrt 12), the RMS error of one uniformly coded
+ *       angle; an evicted token costs eps = 1 (its whole logit is lost);
+ *   R16 rate R(b) = H_kv (16 b + 1 + 256) bytes for a resident token (codes,
+ *       radius byte, bf16 value row), 0 when evicted;
+ *   R17 protected tokens take b_max (the largest tier allowed) and count
+ *       against the budget.
+ * Solver (the Lagrangian relaxation): every token minimises
+ * D_t(b) + lambda R(b) on its own (equal costs: the larger b); lambda is the
+ * smallest value, found by doubling then 100 bisection steps, whose total
+ * rate fits the budget.  Returns 0, or 1 when the protected tokens alone
+ * exceed the budget (then all others are evicted).  keys [T, H_kv, d] bf16;
+ * qn [H_kv]; protect [T] or NULL; tier_mask bit t: b = {3,4,6,8}[t]. */
+static const int kRdrBits[4] = {3, 4, 6, 8};
+
+static double rdr_eps(int b) { return b == 0 ? 1.0 : SPKV_ORACLE_PI / (ldexp(1.0, b) * sqrt(12.0)); }
+
+static double rdr_rate(int b, int Hkv) { return b == 0 ? 0.0 : (double)Hkv * (16.0 * b + 1.0 + 256.0); }
+
+static double rdr_assign(int T, int Hkv, const double *w, const uint8_t *protect, uint32_t tier_mask, int bmax,
+                         double lambda, int32_t *tier)
+{
+    double rate = 0.0;
+    for (int t = 0; t < T; ++t) {
+        int best = 0;
+        if (protect && protect[t]) {
+            best = bmax;
+        } else {
+            double bc = w[t] * rdr_eps(0) + lambda * rdr_rate(0, Hkv);
+            for (int i = 0; i < 4; ++i) {
+                if (!((tier_mask >> i) & 1u)) continue;
+                const int b = kRdrBits[i];
+                const double c = w[t] * rdr_eps(b) + lambda * rdr_rate(b, Hkv);
+                if (c <= bc) { bc = c; best = b; }
+            }
+        }
+        tier[t] = best;
+        rate += rdr_rate(best, Hkv);
+    }
+    return rate;
+}
+
+int spkv_oracle_rdr_plan(int d, int T, int Hkv, const uint16_t *keys, const double *qn, const uint8_t *protect,
+                         double budget, uint32_t tier_mask, int32_t *tier, double *lambda_out, double *rate_out,
+                         double *dist_out)
+{
+    int bmax = 0, status = 0;
+    for (int i = 0; i < 4; ++i)
+        if ((tier_mask >> i) & 1u) bmax = kRdrBits[i];
+    double *w = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    for (int t = 0; t < T; ++t) {
+        double wt = 0.0;
+        for (int h = 0; h < Hkv; ++h) {
+            double n2 = 0.0;
+            for (int j = 0; j < d; ++j) {
+                const double x = spkv_oracle_bf16_to_f64(keys[((size_t)t * Hkv + h) * d + j]);
+                n2 += x * x;
+            }
+            wt += qn[h] * sqrt(n2);
+        }
+        w[t] = wt;
+    }
+    double lambda = 0.0;
+    double rate = rdr_assign(T, Hkv, w, protect, tier_mask, bmax, 0.0, tier);
+    if (rate > budget) {
+        /* lambda large enough that every unprotected token is evicted */
+        double hi = 1.0;
+        int n = 0;
+        while (rdr_assign(T, Hkv, w, protect, tier_mask, bmax, hi, tier) > budget && n < 2000) {
+            hi *= 2.0;
+            ++n;
+        }
+        if (rdr_assign(T, Hkv, w, protect, tier_mask, bmax, hi, tier) > budget) {
+            status = 1; /* the protected tokens alone exceed the budget */
+        } else {
+            double lo = 0.0;
+            for (int it = 0; it < 100; ++it) {
+                const double mid = 0.5 * (lo + hi);
+                if (rdr_assign(T, Hkv, w, protect, tier_mask, bmax, mid, tier) > budget) lo = mid;
+                else hi = mid;
+            }
+        }
+        lambda = hi;
+        rate = rdr_assign(T, Hkv, w, protect, tier_mask, bmax, lambda, tier);
+    }
+    double dist = 0.0;
+    for (int t = 0; t < T; ++t) dist += w[t] * rdr_eps(tier[t]);
+    if (lambda_out) *lambda_out = lambda;
+    if (rate_out) *rate_out = rate;
+    if (dist_out) *dist_out = dist;
+    free(w);
+    return status;
+}

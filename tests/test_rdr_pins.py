@@ -1,0 +1,123 @@
+"""Pins of the oracle's RDR controller (technical summary section 2.2,
+readings R14-R17 in oracle/spkv_oracle.c).
+
+The Lagrangian solve is pinned by brute force (no allocation with at most the
+chosen rate has less surrogate distortion: Everett's theorem for the
+multiplier found), the surrogate's eps_b by a Monte-Carlo RMS of the actual
+angle quantiser, and the budget / protection rules by their definitions."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+
+OPTIONS = (0, 3, 4, 6, 8)
+
+
+def _keys(rng, T, H, d, scale=None):
+    import torch
+
+    x = rng.standard_normal((T, H, d)) * (scale if scale is not None else rng.lognormal(0, 0.7, (T, H, 1)))
+    return torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _w(keys, qn):
+    kf = oracle.bf16_to_f64(keys)
+    return (np.linalg.norm(kf, axis=2) * np.asarray(qn)[None, :]).sum(axis=1)
+
+
+def _eps(b):
+    return 1.0 if b == 0 else math.pi / (2 ** b * math.sqrt(12.0))
+
+
+def _rate(b, H):
+    return 0.0 if b == 0 else H * (16 * b + 1 + 256)
+
+
+def test_eps_is_the_rms_error_of_the_angle_quantiser():
+    rng = np.random.default_rng(1)
+    phi = rng.uniform(0, math.pi, 200_000)
+    for b in (3, 4, 6, 8):
+        mids = np.array([oracle.angle_mid(oracle.angle_code(p, b, 0), b, 0) for p in phi[:20000]])
+        rms = math.sqrt(np.mean((phi[:20000] - mids) ** 2))
+        assert abs(rms / _eps(b) - 1.0) < 0.02, (b, rms, _eps(b))
+
+
+@pytest.mark.parametrize("seed", [2, 3, 4])
+def test_lagrangian_allocation_is_optimal_for_its_rate(seed):
+    rng = np.random.default_rng(seed)
+    T, H, d = 5, 2, 8
+    keys = _keys(rng, T, H, d)
+    qn = rng.uniform(0.5, 2.0, H)
+    protect = np.zeros(T, np.uint8)
+    protect[rng.integers(T)] = 1
+    w = _w(keys, qn)
+    full = T * _rate(8, H)
+    for frac in (0.25, 0.4, 0.6, 0.85):  # (one protected token at b = 8 is 0.2 of full)
+        tiers, lam, rate, dist, st = oracle.rdr_plan(keys, qn, frac * full, protect=protect)
+        assert st == 0 and rate <= frac * full
+        assert dist == pytest.approx(sum(w[t] * _eps(int(tiers[t])) for t in range(T)), rel=1e-12)
+        assert rate == sum(_rate(int(b), H) for b in tiers)
+        best = math.inf
+        for choice in itertools.product(OPTIONS, repeat=T):
+            if any(protect[t] and choice[t] != 8 for t in range(T)):
+                continue
+            r = sum(_rate(b, H) for b in choice)
+            if r <= rate:
+                best = min(best, sum(w[t] * _eps(choice[t]) for t in range(T)))
+        assert dist <= best * (1 + 1e-12), (dist, best)
+
+
+def test_budget_protection_and_limits():
+    rng = np.random.default_rng(5)
+    T, H, d = 64, 4, 32
+    keys = _keys(rng, T, H, d)
+    qn = np.ones(H)
+    protect = np.zeros(T, np.uint8)
+    protect[:4] = 1
+    full = T * _rate(8, H)
+    # everything fits: all at b_max, lambda = 0
+    tiers, lam, rate, dist, st = oracle.rdr_plan(keys, qn, full, protect=protect)
+    assert st == 0 and lam == 0.0 and np.all(tiers == 8)
+    # tier mask {3, 4}: b_max = 4
+    tiers, lam, rate, dist, st = oracle.rdr_plan(keys, qn, full, tier_mask=0x3, protect=protect)
+    assert np.all(tiers == 4)
+    # a tight budget: protected at b_max, the rest fits
+    budget = 0.3 * full
+    tiers, lam, rate, dist, st = oracle.rdr_plan(keys, qn, budget, protect=protect)
+    assert st == 0 and rate <= budget and np.all(tiers[:4] == 8) and lam > 0
+    # only the protected tokens fit: every other token evicted
+    tiers, lam, rate, dist, st = oracle.rdr_plan(keys, qn, 4 * _rate(8, H), protect=protect)
+    assert st == 0 and np.all(tiers[:4] == 8) and np.all(tiers[4:] == 0)
+    # infeasible: the protected tokens alone exceed the budget
+    tiers, lam, rate, dist, st = oracle.rdr_plan(keys, qn, 3 * _rate(8, H), protect=protect)
+    assert st == 1 and np.all(tiers[:4] == 8) and np.all(tiers[4:] == 0)
+
+
+def test_distortion_falls_as_the_budget_grows():
+    rng = np.random.default_rng(6)
+    keys = _keys(rng, 200, 4, 32)
+    qn = rng.uniform(0.5, 2.0, 4)
+    full = 200 * _rate(8, 4)
+    prev_d, prev_r = math.inf, -1.0
+    for frac in np.linspace(0.05, 1.0, 12):
+        _, _, rate, dist, st = oracle.rdr_plan(keys, qn, frac * full)
+        assert st == 0 and rate <= frac * full
+        assert dist <= prev_d * (1 + 1e-12) and rate >= prev_r
+        prev_d, prev_r = dist, rate
+
+
+def test_high_weight_tokens_are_kept_first():
+    """With equal rates per tier, the surrogate orders tokens by w_t: under a
+    budget for half the tokens, every kept token weighs at least every evicted one."""
+    rng = np.random.default_rng(7)
+    T, H = 40, 2
+    keys = _keys(rng, T, H, 16)
+    qn = np.ones(H)
+    tiers, _, _, _, st = oracle.rdr_plan(keys, qn, T / 2 * _rate(4, H), tier_mask=0x2)
+    w = _w(keys, qn)
+    kept, evicted = w[tiers > 0], w[tiers == 0]
+    assert st == 0 and len(kept) and len(evicted)
+    assert kept.min() >= evicted.max()
