@@ -35,10 +35,10 @@ _p = ctypes.c_void_p
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (-O2, no fast-math) into oracle/libspkv_oracle.so."""
+    """Compile the oracle with gcc (-O2, no fast-math, no FMA contraction) into oracle/libspkv_oracle.so."""
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + ".tmp%d" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off",
                                "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -267,3 +267,30 @@ def rdr_plan(keys_bf16, q_norms, budget_bytes, tier_mask=0xF, protect=None):
     st = lib().spkv_oracle_rdr_plan(d, T, Hkv, _ptr(k), _ptr(qn), _ptr(pr), float(budget_bytes), int(tier_mask),
                                     _ptr(tiers), ctypes.byref(lam), ctypes.byref(rate), ctypes.byref(dist))
     return tiers, lam.value, rate.value, dist.value, int(st)
+
+
+RDR_TIER_ORDER = (3, 4, 6, 8)
+
+
+def rdr_pack(tiers, page=16):
+    """Tier-homogeneous pages for a plan (section 2.2: every page holds one
+    precision tier).  Reading: the resident tokens are grouped by tier in
+    ascending b, ascending t within a tier, and each group fills whole pages
+    of 16 slots (its last page partly); attention over the kept tokens does
+    not depend on their order, since keys are stored after RoPE.
+
+    Returns (dst_pos [T] int32: page * 16 + slot in the packed sequence, -1
+    when evicted; page_bits [n_pages] uint8; page_keep [n_pages] uint16, bit s
+    set when slot s holds a token)."""
+    tiers = np.asarray(tiers).reshape(-1)
+    dst = np.full(tiers.shape[0], -1, np.int32)
+    bits, keep = [], []
+    for b in RDR_TIER_ORDER:
+        toks = [t for t in range(tiers.shape[0]) if int(tiers[t]) == b]
+        for r, t in enumerate(toks):
+            dst[t] = len(bits) * page + r
+        for p0 in range(0, len(toks), page):
+            n = min(page, len(toks) - p0)
+            bits.append(b)
+            keep.append((1 << n) - 1)
+    return dst, np.array(bits, np.uint8), np.array(keep, np.uint16)

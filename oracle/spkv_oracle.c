@@ -384,7 +384,7 @@ void spkv_oracle_dense_group(int d, int G, int T, const uint16_t *q, const uint1
  * D_t(b) + lambda R(b) on its own (equal costs: the larger b); lambda is the
  * smallest value, found by doubling then 100 bisection steps, whose total
  * rate fits the budget.  Returns 0, or 1 when the protected tokens alone
- * exceed the budget (then all others are evicted).  keys [T, H_kv, d] bf16;
+ * exceed the budget (then all others are evicted and lambda = +inf).  keys [T, H_kv, d] bf16;
  * qn [H_kv]; protect [T] or NULL; tier_mask bit t: b = {3,4,6,8}[t]. */
 static const int kRdrBits[4] = {3, 4, 6, 8};
 
@@ -438,25 +438,34 @@ int spkv_oracle_rdr_plan(int d, int T, int Hkv, const uint16_t *keys, const doub
     double lambda = 0.0;
     double rate = rdr_assign(T, Hkv, w, protect, tier_mask, bmax, 0.0, tier);
     if (rate > budget) {
-        /* lambda large enough that every unprotected token is evicted */
-        double hi = 1.0;
-        int n = 0;
-        while (rdr_assign(T, Hkv, w, protect, tier_mask, bmax, hi, tier) > budget && n < 2000) {
-            hi *= 2.0;
-            ++n;
-        }
-        if (rdr_assign(T, Hkv, w, protect, tier_mask, bmax, hi, tier) > budget) {
-            status = 1; /* the protected tokens alone exceed the budget */
+        double prot_rate = 0.0;
+        for (int t = 0; t < T; ++t)
+            if (protect && protect[t]) prot_rate += rdr_rate(bmax, Hkv);
+        if (prot_rate > budget) {
+            /* the protected tokens alone exceed the budget: no multiplier
+             * fits; they stay at b_max and every other token is evicted */
+            status = 1;
+            lambda = INFINITY;
+            for (int t = 0; t < T; ++t) tier[t] = (protect && protect[t]) ? bmax : 0;
+            rate = prot_rate;
         } else {
+            /* a multiplier large enough that the rate fits (at worst every
+             * unprotected token evicted), then bisection on [0, hi] */
+            double hi = 1.0;
+            int n = 0;
+            while (rdr_assign(T, Hkv, w, protect, tier_mask, bmax, hi, tier) > budget && n < 2000) {
+                hi *= 2.0;
+                ++n;
+            }
             double lo = 0.0;
             for (int it = 0; it < 100; ++it) {
                 const double mid = 0.5 * (lo + hi);
                 if (rdr_assign(T, Hkv, w, protect, tier_mask, bmax, mid, tier) > budget) lo = mid;
                 else hi = mid;
             }
+            lambda = hi;
+            rate = rdr_assign(T, Hkv, w, protect, tier_mask, bmax, lambda, tier);
         }
-        lambda = hi;
-        rate = rdr_assign(T, Hkv, w, protect, tier_mask, bmax, lambda, tier);
     }
     double dist = 0.0;
     for (int t = 0; t < T; ++t) dist += w[t] * rdr_eps(tier[t]);

@@ -121,3 +121,34 @@ def test_high_weight_tokens_are_kept_first():
     kept, evicted = w[tiers > 0], w[tiers == 0]
     assert st == 0 and len(kept) and len(evicted)
     assert kept.min() >= evicted.max()
+
+
+def test_infeasible_plan_reports_an_infinite_multiplier():
+    rng = np.random.default_rng(8)
+    keys = _keys(rng, 10, 2, 16)
+    protect = np.ones(10, np.uint8)
+    tiers, lam, rate, _, st = oracle.rdr_plan(keys, np.ones(2), 9 * _rate(8, 2), protect=protect)
+    assert st == 1 and lam == math.inf and np.all(tiers == 8) and rate == 10 * _rate(8, 2)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_pack_makes_tier_homogeneous_pages(seed):
+    """Every resident token lands in exactly one slot of a page of its own
+    tier; pages are grouped by ascending tier; the keep bits are the occupied
+    slots; a group of n tokens takes ceil(n / 16) pages."""
+    rng = np.random.default_rng(seed)
+    T = int(rng.integers(1, 300))
+    tiers = rng.choice(OPTIONS, size=T, p=[0.2, 0.2, 0.3, 0.2, 0.1])
+    dst, bits, keep = oracle.rdr_pack(tiers)
+    assert np.all((dst < 0) == (tiers == 0))
+    kept = dst[dst >= 0]
+    assert len(np.unique(kept)) == len(kept)
+    occupied = np.zeros((len(bits), 16), bool)
+    occupied[kept // 16, kept % 16] = True
+    for p in range(len(bits)):
+        assert keep[p] == sum(1 << s for s in range(16) if occupied[p, s])
+    assert np.all(bits[dst[tiers > 0] // 16] == tiers[tiers > 0])
+    assert np.all(np.diff(bits.astype(int)) >= 0)
+    assert len(bits) == sum(-(-int(np.sum(tiers == b)) // 16) for b in (3, 4, 6, 8))
+    for b in (3, 4, 6, 8):  # ascending t within a tier
+        assert np.all(np.diff(dst[tiers == b]) > 0)
