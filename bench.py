@@ -343,6 +343,19 @@ def compare_paths(args, spkv, workload, wl, cache, ctx, max_ctx, splits, ws, str
     res["encode_unit"] = "(token, kv head) keys/s, with values"
     res["resident_bytes_per_token"] = {"ada": cache.resident_bytes() / tokens,
                                        "dense_bf16": 2 * wl.Hkv * 256.0}
+    # RDR controller (weights kernel + one cluster per sequence) over the
+    # batch's context keys: 35% of the b = 8 bytes, sinks + last 64 protected
+    ri = synthetic.make_rdr_inputs(wl, budget_frac=0.35)
+    seq = torch.from_numpy(ri.seq_start).to(dev)
+    qn = torch.from_numpy(ri.q_norms).to(dev)
+    bud = torch.from_numpy(ri.budget).to(dev)
+    prot = torch.from_numpy(ri.protect).to(dev)
+    ntok = int(wl.keys.shape[0])
+    rws = torch.empty(spkv.rdr_workspace_bytes(ntok), dtype=torch.uint8, device=dev)
+    rdr_ms = timeit(lambda: spkv.rdr_plan(wl.keys, seq, qn, bud, protect=prot, ws=rws, stream=stream))
+    res["rdr_plan_ms"] = rdr_ms
+    res["rdr_plan_tokens_per_s"] = ntok / (rdr_ms * 1e-3)
+    res["rdr_plan_key_bytes_gbs"] = wl.keys.numel() * 2 / (rdr_ms * 1e-3) / 1e9
     return res
 
 

@@ -34,10 +34,14 @@ EXPORTS = (
     "spkv_decode_attention_partial",
     "spkv_merge_partials",
     "spkv_debug_wait_timeout",
+    "spkv_rdr_workspace_bytes",
+    "spkv_rdr_plan",
+    "spkv_encode_keys_packed",
 )
 PARTIAL_FLOATS = 132  # floats per (sequence, query head) shard record
 DECODE_EXACT_Q = 1  # SPKV_DECODE_EXACT_Q
 STATIC_WS_BYTES = 16 * 1024 * 1024  # SPKV_STATIC_WS_BYTES
+RDR_INFEASIBLE, RDR_PAGES, RDR_BAD_RANGE = 1, 2, 4  # SPKV_RDR_* status bits
 
 
 class SpkvError(RuntimeError):
@@ -114,6 +118,14 @@ def _load():
     L.spkv_debug_logits_ex.restype = ctypes.c_int
     L.spkv_debug_logits_ex.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _I, _I, _P, _I, _P, _I, _P, ctypes.c_uint32,
                                        _P]
+    L.spkv_rdr_workspace_bytes.restype = ctypes.c_size_t
+    L.spkv_rdr_workspace_bytes.argtypes = [ctypes.c_int64]
+    L.spkv_rdr_plan.restype = ctypes.c_int
+    L.spkv_rdr_plan.argtypes = [_P, _P, _I, ctypes.c_int64, _I, _P, _P, _P, ctypes.c_uint32, _I, _P, _P, _P, _P,
+                                _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    L.spkv_encode_keys_packed.restype = ctypes.c_int
+    L.spkv_encode_keys_packed.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _P, _P, _I, ctypes.c_int64, _P, _P, _I,
+                                          _P]
     return L
 
 

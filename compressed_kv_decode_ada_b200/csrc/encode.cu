@@ -34,8 +34,9 @@ struct EncodeParams {
   int Hkv, num_pages;
   const uint16_t *keys, *values;
   const int32_t *start_pos, *block_table;
+  const int32_t *seq_start, *dst_pos;  // scattered placement (start_pos unused)
   int B, n_new, max_pages;
-  int64_t items;  // B * n_new * Hkv
+  int64_t items;  // B * n_new * Hkv, or total_tokens * Hkv when scattered
 };
 
 struct EncodeSmem {
@@ -54,9 +55,25 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams 
   for (int64_t item = (int64_t)blockIdx.x * kEncWarps + wid; item < p.items; item += nwarps) {
     const int h = (int)(item % p.Hkv);
     const int64_t bn = item / p.Hkv;
-    const int b = (int)(bn / p.n_new);
-    const int n = (int)(bn % p.n_new);
-    const int pos = p.start_pos[b] + n;
+    int b, pos;
+    if (p.dst_pos) {  // token bn of the concatenated sequences, to dst_pos[bn]
+      pos = p.dst_pos[bn];
+      if (pos < 0) continue;
+      int lo = 0, hi = p.B;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)p.seq_start[mid] <= bn) lo = mid;
+        else hi = mid;
+      }
+      b = lo;
+      if (bn < (int64_t)p.seq_start[b] || bn >= (int64_t)p.seq_start[b + 1]) {
+        if (lane == 0) set_err(p.err, SPKV_DEVERR_CTX);
+        continue;
+      }
+    } else {
+      b = (int)(bn / p.n_new);
+      pos = p.start_pos[b] + (int)(bn % p.n_new);
+    }
     if (pos < 0 || pos >= p.max_pages * kPage) {
       if (lane == 0) set_err(p.err, SPKV_DEVERR_CTX);
       continue;
@@ -109,6 +126,30 @@ int device_sm_count();
 
 }  // namespace spkv
 
+namespace spkv {
+namespace {
+
+spkv_status launch_encode(const spkv_cache *cache, EncodeParams &p, cudaStream_t stream) {
+  p.arena = cache->code_arena;
+  p.arena_bytes = cache->code_arena_bytes;
+  p.hdr = cache->hdr;
+  p.rad_lo = cache->rad_lo_log2;
+  p.rad_step = cache->rad_step_log2;
+  p.v_pages = cache->v_pages;
+  p.err = cache->err_flags;
+  p.Hkv = cache->num_kv_heads;
+  p.num_pages = cache->num_pages;
+  const int sms = device_sm_count();
+  if (sms <= 0) return SPKV_ERR_CUDA;
+  const int64_t want = (p.items + kEncWarps - 1) / kEncWarps;
+  const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+  encode_kernel<<<grid, kEncThreads, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace spkv
+
 extern "C" spkv_status spkv_encode_keys(const spkv_cache *cache, const uint16_t *keys, const uint16_t *values,
                                         const int32_t *start_pos, int32_t B, int32_t n_new,
                                         const int32_t *block_table, int32_t max_pages, void *stream) {
@@ -119,16 +160,7 @@ extern "C" spkv_status spkv_encode_keys(const spkv_cache *cache, const uint16_t 
   if (B == 0 || n_new == 0) return SPKV_OK;
   if (!keys || !start_pos || !block_table || max_pages == 0) return SPKV_ERR_INVALID_ARG;
   if (((uintptr_t)keys & 7) || ((uintptr_t)values & 7)) return SPKV_ERR_INVALID_ARG;
-  EncodeParams p;
-  p.arena = cache->code_arena;
-  p.arena_bytes = cache->code_arena_bytes;
-  p.hdr = cache->hdr;
-  p.rad_lo = cache->rad_lo_log2;
-  p.rad_step = cache->rad_step_log2;
-  p.v_pages = cache->v_pages;
-  p.err = cache->err_flags;
-  p.Hkv = cache->num_kv_heads;
-  p.num_pages = cache->num_pages;
+  EncodeParams p = {};
   p.keys = keys;
   p.values = values;
   p.start_pos = start_pos;
@@ -137,10 +169,29 @@ extern "C" spkv_status spkv_encode_keys(const spkv_cache *cache, const uint16_t 
   p.n_new = n_new;
   p.max_pages = max_pages;
   p.items = (int64_t)B * n_new * cache->num_kv_heads;
-  const int sms = device_sm_count();
-  if (sms <= 0) return SPKV_ERR_CUDA;
-  const int64_t want = (p.items + kEncWarps - 1) / kEncWarps;
-  const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
-  encode_kernel<<<grid, kEncThreads, 0, (cudaStream_t)stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
+  return launch_encode(cache, p, (cudaStream_t)stream);
+}
+
+extern "C" spkv_status spkv_encode_keys_packed(const spkv_cache *cache, const uint16_t *keys, const uint16_t *values,
+                                               const int32_t *seq_start, int32_t B, int64_t total_tokens,
+                                               const int32_t *dst_pos, const int32_t *block_table, int32_t max_pages,
+                                               void *stream) {
+  using namespace spkv;
+  spkv_status st = check_cache(cache);
+  if (st != SPKV_OK) return st;
+  if (B < 0 || total_tokens < 0 || max_pages < 0) return SPKV_ERR_INVALID_ARG;
+  if (B == 0 || total_tokens == 0) return SPKV_OK;
+  if (!keys || !seq_start || !dst_pos || !block_table || max_pages == 0) return SPKV_ERR_INVALID_ARG;
+  if (((uintptr_t)keys & 7) || ((uintptr_t)values & 7)) return SPKV_ERR_INVALID_ARG;
+  EncodeParams p = {};
+  p.keys = keys;
+  p.values = values;
+  p.seq_start = seq_start;
+  p.dst_pos = dst_pos;
+  p.block_table = block_table;
+  p.B = B;
+  p.n_new = 0;
+  p.max_pages = max_pages;
+  p.items = total_tokens * cache->num_kv_heads;
+  return launch_encode(cache, p, (cudaStream_t)stream);
 }

@@ -237,3 +237,73 @@ def debug_logits(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tensor, c
                                    _ptr(ctx_lens), int(max_ctx), _ptr(logits), DECODE_EXACT_Q if exact_q else 0,
                                    _stream(stream)), "spkv_debug_logits_ex")
     return logits
+
+
+def encode_keys_packed(cache: SpkvCache, keys: torch.Tensor, seq_start: torch.Tensor, dst_pos: torch.Tensor,
+                       block_table: torch.Tensor, values: torch.Tensor | None = None, stream=None) -> None:
+    """spkv_encode_keys_packed: keys/values [total_tokens, H_kv, 128] bf16, token t of sequence s
+    to position dst_pos[t] of s (negative: skipped)."""
+    _need(keys, torch.bfloat16, "keys", 3)
+    total, hkv, d = keys.shape
+    if hkv != cache.num_kv_heads or d != HEAD_DIM:
+        raise ValueError("keys must be [total_tokens, H_kv, 128]")
+    if values is not None:
+        _need(values, torch.bfloat16, "values", 3)
+        if values.shape != keys.shape:
+            raise ValueError("values must match keys")
+    _need(seq_start, torch.int32, "seq_start", 1)
+    _need(dst_pos, torch.int32, "dst_pos", 1)
+    _need(block_table, torch.int32, "block_table", 2)
+    B = seq_start.shape[0] - 1
+    if dst_pos.shape[0] != total or block_table.shape[0] != B:
+        raise ValueError("dst_pos / block_table shape mismatch")
+    c = cache.c_struct()
+    check(lib.spkv_encode_keys_packed(ctypes.byref(c), _ptr(keys), _ptr(values), _ptr(seq_start), B, total,
+                                      _ptr(dst_pos), _ptr(block_table), block_table.shape[1], _stream(stream)),
+          "spkv_encode_keys_packed")
+
+
+def rdr_workspace_bytes(total_tokens: int) -> int:
+    return int(lib.spkv_rdr_workspace_bytes(int(total_tokens)))
+
+
+def rdr_plan(keys: torch.Tensor, seq_start: torch.Tensor, q_norms: torch.Tensor, budget_bytes: torch.Tensor,
+             protect: torch.Tensor | None = None, tier_mask: int = 0xF, max_pages_out: int | None = None,
+             ws: torch.Tensor | None = None, stream=None) -> dict:
+    """spkv_rdr_plan over sequences concatenated in keys [total_tokens, H_kv, 128] bf16.
+
+    Returns a dict of device tensors: tier [T] uint8, dst_pos [T] int32,
+    page_bits / page_keep [B, max_pages_out], n_pages [B] int32, lambda,
+    rate, dist [B] float64, status [B] int32."""
+    _need(keys, torch.bfloat16, "keys", 3)
+    total, hkv, d = keys.shape
+    if d != HEAD_DIM:
+        raise ValueError("keys must be [total_tokens, H_kv, 128]")
+    _need(seq_start, torch.int32, "seq_start", 1)
+    B = seq_start.shape[0] - 1
+    _need(q_norms, torch.float32, "q_norms", 2)
+    _need(budget_bytes, torch.float64, "budget_bytes", 1)
+    if tuple(q_norms.shape) != (B, hkv) or budget_bytes.shape[0] != B:
+        raise ValueError("q_norms must be [B, H_kv] and budget_bytes [B]")
+    if protect is not None:
+        _need(protect, torch.uint8, "protect", 1)
+        if protect.shape[0] != total:
+            raise ValueError("protect must be [total_tokens]")
+    dev = keys.device
+    if max_pages_out is None:
+        max_pages_out = (total + 15) // 16 + 3
+    if ws is None:
+        ws = torch.empty(rdr_workspace_bytes(total), dtype=torch.uint8, device=dev)
+    out = dict(tier=torch.empty(total, dtype=torch.uint8, device=dev),
+               dst_pos=torch.empty(total, dtype=torch.int32, device=dev),
+               page_bits=torch.zeros((B, max(max_pages_out, 1)), dtype=torch.uint8, device=dev),
+               page_keep=torch.zeros((B, max(max_pages_out, 1)), dtype=torch.int16, device=dev),
+               n_pages=torch.empty(B, dtype=torch.int32, device=dev),
+               **{k: torch.empty(B, dtype=torch.float64, device=dev) for k in ("lambda", "rate", "dist")},
+               status=torch.empty(B, dtype=torch.int32, device=dev))
+    check(lib.spkv_rdr_plan(_ptr(keys), _ptr(seq_start), B, total, hkv, _ptr(q_norms), _ptr(protect),
+                            _ptr(budget_bytes), int(tier_mask), int(max_pages_out), _ptr(out["tier"]),
+                            _ptr(out["dst_pos"]), _ptr(out["page_bits"]), _ptr(out["page_keep"]),
+                            _ptr(out["n_pages"]), _ptr(out["lambda"]), _ptr(out["rate"]), _ptr(out["dist"]),
+                            _ptr(out["status"]), _ptr(ws), ws.numel(), _stream(stream)), "spkv_rdr_plan")
+    return out

@@ -259,3 +259,38 @@ def dense_step_bytes(wl: Workload) -> float:
     plus 4/16 bytes of block table per token."""
     n = float(wl.ctx.sum())
     return n * (512.0 * wl.Hkv + 0.25)
+
+
+@dataclass
+class RdrInputs:
+    """Inputs of the RDR controller for the sequences of a workload."""
+    seq_start: np.ndarray  # [B + 1] int32 (the workload's seq_off)
+    q_norms: np.ndarray    # [B, H_kv] float32
+    protect: np.ndarray    # [ntok] uint8
+    budget: np.ndarray     # [B] float64 bytes
+
+
+def make_rdr_inputs(wl: Workload, budget_frac: float = 0.35, sinks: int = 4, recent: int = 64,
+                    seed: int | None = None) -> RdrInputs:
+    """Seeded RDR inputs for a workload's keys (section 2.2's controller):
+
+      q_norms  per (sequence, kv head) ~ sqrt(128) * LogNormal(0, 0.25), the
+               magnitude of a 128-d standard normal query, as fp32;
+      protect  the first `sinks` tokens (attention sinks) and the last
+               `recent` tokens (the local window) of every sequence;
+      budget   budget_frac x the bytes of the whole sequence at b = 8
+               (T * H_kv * (16 * 8 + 1 + 256)).
+    """
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(wl.seed if seed is None else seed) + 7919)
+    qn = (math.sqrt(HEAD_DIM) * torch.exp(0.25 * torch.randn((wl.B, wl.Hkv), generator=gen,
+                                                             dtype=torch.float64))).numpy().astype(np.float32)
+    ntok = int(wl.seq_off[-1])
+    protect = np.zeros(ntok, np.uint8)
+    for b in range(wl.B):
+        s0, s1 = int(wl.seq_off[b]), int(wl.seq_off[b + 1])
+        protect[s0:min(s1, s0 + sinks)] = 1
+        protect[max(s0, s1 - recent):s1] = 1
+    full = wl.ctx.astype(np.float64) * wl.Hkv * (16 * 8 + 1 + 256)
+    return RdrInputs(seq_start=wl.seq_off.astype(np.int32), q_norms=qn, protect=protect,
+                     budget=np.floor(budget_frac * full))

@@ -305,6 +305,82 @@ SPKV_API spkv_status spkv_debug_logits_ex(const spkv_cache *cache, const uint16_
  * counterpart: this checks the library's own failure handling.) */
 SPKV_API spkv_status spkv_debug_wait_timeout(uint32_t *err_flags, int32_t *status, uint64_t limit_ns, void *stream);
 
+/* ------------------------------------------------------------------ RDR
+ * Rate-distortion retention controller (technical summary section 2.2: a
+ * residency decision and a precision tier for every state under a hard
+ * memory budget, from a distortion surrogate built on the codes' angular
+ * error scaled by query and key magnitudes; protected states at the top
+ * tier; tier-homogeneous pages).  Readings, for the parts the section leaves
+ * open:
+ *   - the unit is a token: its kv heads share a page and so a tier;
+ *   - D_t(b) = w_t eps_b, w_t = sum_h qn_h ||k_{t,h}||_2, eps_b =
+ *     pi / (2^b sqrt 12); an evicted token costs w_t (eps = 1);
+ *   - rate R(b) = H_kv (16 b + 1 + 256) bytes for a resident token (angle
+ *     codes, radius byte, bf16 value row), 0 when evicted;
+ *   - protected tokens take b_max, the largest tier in tier_mask.
+ * Each token minimises D_t(b) + lambda R(b) (ties: the larger b); lambda is
+ * the smallest multiplier whose total rate fits the budget, found by doubling
+ * from 1 and bisection on [0, hi] in fp64 (at most 100 halvings).  The plan
+ * is then packed: resident tokens grouped by tier (b ascending), ascending t
+ * within a tier, each group filling whole pages of 16 slots, its last page
+ * partly (attention over the kept tokens does not depend on their order).
+ *
+ *   keys        [total_tokens, H_kv, 128] bf16, device, 16-byte aligned:
+ *               sequence s owns rows seq_start[s] .. seq_start[s+1]-1
+ *   seq_start   [B + 1] int32, device, nondecreasing, in [0, total_tokens]
+ *   q_norms     [B, H_kv] fp32, device: qn_h per sequence (>= 0)
+ *   protect     [total_tokens] uint8, device, or NULL: nonzero = protected
+ *   budget_bytes [B] fp64, device: the rate budget of each sequence
+ *   tier_mask   allowed tiers, bit i: b = {3,4,6,8}[i]; nonzero, < 16
+ *   max_pages_out  capacity of page_bits / page_keep per sequence; a plan
+ *               needs at most ceil(T_s / 16) + 3 pages
+ * Outputs (device):
+ *   tier        [total_tokens] uint8: b, or 0 = evicted
+ *   dst_pos     [total_tokens] int32: page * 16 + slot of the token in its
+ *               sequence's packed pages, -1 when evicted
+ *   page_bits   [B, max_pages_out] uint8: b of packed page p (p < n_pages)
+ *   page_keep   [B, max_pages_out] uint16: occupied slots of packed page p
+ *   n_pages     [B] int32: packed pages of the sequence
+ *   lambda, rate_bytes, distortion  [B] fp64: the multiplier (+inf when
+ *               infeasible), the plan's rate and its surrogate distortion
+ *   status      [B] int32: 0, or SPKV_RDR_* bits
+ * ws: spkv_rdr_workspace_bytes(total_tokens) bytes of device memory, 16-byte
+ * aligned, owned by the caller (the per-token weights).  Every pointer is
+ * the caller's; the call only enqueues work on `stream`.  Argument errors
+ * (NULL, misalignment, H_kv outside 1..32, a bad tier_mask, a short
+ * workspace) return without launching. */
+#define SPKV_RDR_INFEASIBLE 0x1 /* protected tokens alone exceed the budget:
+                                   they are kept at b_max, all others evicted */
+#define SPKV_RDR_PAGES 0x2      /* the packed plan needs more than max_pages_out
+                                   pages: n_pages says how many; dst_pos = -1
+                                   and no page entries written */
+#define SPKV_RDR_BAD_RANGE 0x4  /* seq_start out of order or out of range:
+                                   nothing else written for the sequence */
+
+SPKV_API size_t spkv_rdr_workspace_bytes(int64_t total_tokens);
+
+SPKV_API spkv_status spkv_rdr_plan(const uint16_t *keys, const int32_t *seq_start, int32_t B, int64_t total_tokens,
+                                   int32_t num_kv_heads, const float *q_norms, const uint8_t *protect,
+                                   const double *budget_bytes, uint32_t tier_mask, int32_t max_pages_out,
+                                   uint8_t *tier, int32_t *dst_pos, uint8_t *page_bits, uint16_t *page_keep,
+                                   int32_t *n_pages, double *lambda, double *rate_bytes, double *distortion,
+                                   int32_t *status, void *ws, size_t ws_bytes, void *stream);
+
+/* Encode keys (and optionally values) to scattered positions: the packed
+ * layout of an RDR plan (section 2.2) or any other placement.
+ *   keys, values  [total_tokens, H_kv, 128] bf16, device (values may be NULL)
+ *   seq_start     [B + 1] int32, device: sequence s owns rows
+ *                 seq_start[s] .. seq_start[s+1]-1
+ *   dst_pos       [total_tokens] int32, device: position of the token in its
+ *                 sequence (page block_table[s][pos/16], slot pos%16); a
+ *                 negative position skips the token
+ *   block_table   [B, max_pages] int32, device
+ * Codes and errors as spkv_encode_keys. */
+SPKV_API spkv_status spkv_encode_keys_packed(const spkv_cache *cache, const uint16_t *keys, const uint16_t *values,
+                                             const int32_t *seq_start, int32_t B, int64_t total_tokens,
+                                             const int32_t *dst_pos, const int32_t *block_table, int32_t max_pages,
+                                             void *stream);
+
 #ifdef __cplusplus
 }
 #endif
