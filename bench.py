@@ -430,6 +430,45 @@ def cpu_oracle(args, budget_s: float):
                       f"{wl.name} (G={wl.G}, b=4); KV tokens = token-heads / {wl.Hkv}; {dt:.1f} s"}
 
 
+def run_rdr(args):
+    """spkv_rdr_plan (weights kernel + plan kernel) over the workload's context
+    keys: 35% of the b = 8 bytes, sinks + last 64 tokens protected; W warm-up
+    and K timed calls, CUDA events on the launching stream."""
+    import torch
+
+    from compressed_kv_decode_ada_b200 import synthetic
+    import compressed_kv_decode_ada_b200 as spkv
+
+    dev = torch.device("cuda", 0)
+    kw = {"B": args.B} if args.B else {}
+    wl = synthetic.make_workload(args.workload, device=dev, **kw)
+    ri = synthetic.make_rdr_inputs(wl, budget_frac=0.35)
+    seq = torch.from_numpy(ri.seq_start).to(dev)
+    qn = torch.from_numpy(ri.q_norms).to(dev)
+    bud = torch.from_numpy(ri.budget).to(dev)
+    prot = torch.from_numpy(ri.protect).to(dev)
+    ntok = int(wl.keys.shape[0])
+    ws = torch.empty(spkv.rdr_workspace_bytes(ntok), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        plan = spkv.rdr_plan(wl.keys, seq, qn, bud, protect=prot, ws=ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        plan = spkv.rdr_plan(wl.keys, seq, qn, bud, protect=prot, ws=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    weights_bytes = ntok * (wl.Hkv * 256 + 1 + 8)
+    return {"metric": "RDR plan: planned tokens/s", "value": ntok / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "config": {"workload": wl.name, "B": wl.B, "num_kv_heads": wl.Hkv, "tokens": ntok, "budget_frac": 0.35,
+                       "protected": "first 4 + last 64 tokens of each sequence",
+                       "weights_kernel_algorithmic_bytes": weights_bytes},
+            "status": plan["status"].cpu().tolist()[:8], "gpu_launches": 2 * args.steps}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -445,6 +484,8 @@ def main():
     ap.add_argument("--compare-steps", type=int, default=50)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rdr", action="store_true",
+                    help="time only spkv_rdr_plan on the workload's keys (one JSON line; profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -464,6 +505,11 @@ def main():
                 "e2e": {"value": cb["value"], "unit": "KV tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
+        return 0
+
+    if args.rdr:
+        if rank == 0:
+            print(json.dumps(run_rdr(args)), flush=True)
         return 0
 
     res = run_spkv(args, rank, world, local)

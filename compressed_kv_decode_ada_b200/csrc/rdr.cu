@@ -97,7 +97,19 @@ __device__ __forceinline__ double bf16_abs_f64(uint32_t h16) {
 // value is exact in fp64, so n2 + x * x rounded once, an FMA, is the sum of
 // the exact square), and the kv heads of a token are added in ascending
 // order.
-__global__ void __launch_bounds__(kWThreads) rdr_weights_kernel(const WeightParams p) {
+// Halfword-wise unsigned min / max of two words.
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__global__ void __launch_bounds__(kWThreads, 6) rdr_weights_kernel(const WeightParams p) {
   __shared__ uint4 tile[kWWarps][32 * kTileU4];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   uint4 *tl = tile[wid];
@@ -108,32 +120,64 @@ __global__ void __launch_bounds__(kWThreads) rdr_weights_kernel(const WeightPara
     const int rows = ntok * p.Hkv;
     const int nchunks = rows * kRowU4;
     const uint4 *src = reinterpret_cast<const uint4 *>(p.keys) + t0 * p.Hkv * kRowU4;
-    uint4 v[16];
+    // the tile in two rounds of 8 chunks per lane (registers stay under 64)
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int c = lane + 32 * i;
-      if (c < nchunks) v[i] = __ldcs(src + c);  // streamed once: evict-first
-    }
+    for (int r = 0; r < 2; ++r) {
+      uint4 v[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int c = lane + 32 * i;
-      if (c < nchunks) tl[(c >> 4) * kTileU4 + (c & 15)] = v[i];
+      for (int i = 0; i < 8; ++i) {
+        const int c = lane + 32 * (8 * r + i);
+        if (c < nchunks) v[i] = __ldcs(src + c);  // streamed once: evict-first
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = lane + 32 * (8 * r + i);
+        if (c < nchunks) tl[(c >> 4) * kTileU4 + (c & 15)] = v[i];
+      }
     }
     __syncwarp();
     double pr = 0.0;  // qn_h * ||k_{t,h}|| of this lane's row
     const int h = lane % p.Hkv;
     const int64_t t = t0 + lane / p.Hkv;
     if (lane < rows) {
-      double n2 = 0.0;
+      const uint4 *row = tl + lane * kTileU4;
+      // every element of the row a normal bf16 (exponent field 1..254)?
+      uint32_t mn = 0xffffffffu, mx = 0u;
 #pragma unroll 4
       for (int k = 0; k < kRowU4; ++k) {
-        const uint4 q = tl[lane * kTileU4 + k];
-        const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+        const uint4 q = row[k];
+        const uint32_t a0 = q.x & 0x7fff7fffu, a1 = q.y & 0x7fff7fffu, a2 = q.z & 0x7fff7fffu, a3 = q.w & 0x7fff7fffu;
+        mn = min_u16x2(mn, min_u16x2(min_u16x2(a0, a1), min_u16x2(a2, a3)));
+        mx = max_u16x2(mx, max_u16x2(max_u16x2(a0, a1), max_u16x2(a2, a3)));
+      }
+      const bool normal = (mn & 0xffffu) >= 0x0080u && (mn >> 16) >= 0x0080u && (mx & 0xffffu) < 0x7f80u &&
+                          (mx >> 16) < 0x7f80u;
+      double n2 = 0.0;
+      if (normal) {
+        // |x| as fp64: exponent rebiased by 1023 - 127, fraction moved up
+#pragma unroll 4
+        for (int k = 0; k < kRowU4; ++k) {
+          const uint4 q = row[k];
+          const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const double x0 = bf16_abs_f64(wv[e] & 0xffffu), x1 = bf16_abs_f64(wv[e] >> 16);
-          n2 = __fma_rn(x0, x0, n2);
-          n2 = __fma_rn(x1, x1, n2);
+          for (int e = 0; e < 4; ++e) {
+            const double x0 = __hiloint2double((int)((wv[e] & 0x7fffu) * 8192u + 0x38000000u), 0);
+            const double x1 = __hiloint2double((int)(((wv[e] >> 3) & 0x0fffe000u) + 0x38000000u), 0);
+            n2 = __fma_rn(x0, x0, n2);
+            n2 = __fma_rn(x1, x1, n2);
+          }
+        }
+      } else {
+#pragma unroll 2
+        for (int k = 0; k < kRowU4; ++k) {
+          const uint4 q = row[k];
+          const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const double x0 = bf16_abs_f64(wv[e] & 0xffffu), x1 = bf16_abs_f64(wv[e] >> 16);
+            n2 = __fma_rn(x0, x0, n2);
+            n2 = __fma_rn(x1, x1, n2);
+          }
         }
       }
       const int b = seq_of_token(p.seq_start, p.B, t);
@@ -321,15 +365,16 @@ __global__ void __launch_bounds__(kRdrThreads, 1) rdr_plan_kernel(const PlanPara
     // groups of 4 tokens per thread decided without branches; a warp-wide
     // vote sends the (rare) abstentions to fp64.  The trip count is the same
     // for every thread of the CTA (the vote needs all 32 lanes).
-    for (int64_t base = 0; base < nloc; base += 4 * kRdrThreads) {
-      const int64_t j0 = base + tid;
+    const int nl = (int)nloc;  // (< 2^31: seq_start is int32)
+    for (int base = 0; base < nl; base += 4 * kRdrThreads) {
+      const int j0 = base + tid;
       FastDecision d[4];
       bool valid[4];
       float wf[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int64_t j = j0 + (int64_t)u * kRdrThreads;
-        valid[u] = j < nloc;
+        const int j = j0 + u * kRdrThreads;
+        valid[u] = j < nl;
         wf[u] = valid[u] ? wfget(j) : 0.0f;
         d[u] = rdr_choose_fp32(wf[u], p, L);
         d[u].need = d[u].need && valid[u];
@@ -337,7 +382,7 @@ __global__ void __launch_bounds__(kRdrThreads, 1) rdr_plan_kernel(const PlanPara
       if (__any_sync(0xffffffffu, d[0].need || d[1].need || d[2].need || d[3].need)) {
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          if (d[u].need) d[u].i = rdr_choose(wget(j0 + (int64_t)u * kRdrThreads), p, L.r, L.z);
+          if (d[u].need) d[u].i = rdr_choose(wget(j0 + u * kRdrThreads), p, L.r, L.z);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
