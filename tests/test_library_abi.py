@@ -93,3 +93,29 @@ def test_workspace_formula(lib):
     assert lib.workspace_bytes(2, 8, 8, 100, 5) == want(2, 8, 8, 5)
     assert lib.workspace_bytes(3, 8, 1, 100, 5) == want(3, 8, 1, 5)
     assert lib.workspace_bytes(2, 7, 2, 100, 5) == 0  # Hq not a multiple of H_kv
+
+
+def test_rdr_host_argument_checks(lib):
+    """spkv_rdr_plan / spkv_encode_keys_packed reject bad arguments before any
+    CUDA call; an empty batch is a no-op."""
+    L = lib.lib
+    P = 0x10000  # an aligned stand-in pointer, never dereferenced
+
+    def plan(B=2, total=10, Hkv=8, mask=0xF, maxp=8, keys=P, ws=P, ws_bytes=1 << 20, page=P):
+        return L.spkv_rdr_plan(keys, P, B, total, Hkv, P, None, P, mask, maxp, P, P, page, page, P, P, P, P, P,
+                               ws, ws_bytes, None)
+
+    assert plan(Hkv=0) == 1 and plan(Hkv=33) == 1
+    assert plan(mask=0) == 1 and plan(mask=0x10) == 1
+    assert plan(B=-1) == 1 and plan(total=-1) == 1 and plan(maxp=-1) == 1
+    assert plan(keys=P + 8) == 1          # keys must be 16-byte aligned
+    assert plan(page=None) == 1           # page outputs needed when max_pages_out > 0
+    assert plan(ws_bytes=16) == 3         # workspace: 8 bytes per token
+    assert plan(B=0) == 0                 # empty batch
+    assert L.spkv_rdr_workspace_bytes(0) == 16
+    assert L.spkv_rdr_workspace_bytes(1000) == 8000
+    assert L.spkv_rdr_workspace_bytes(1001) == 8016
+    c = _fake_cache(lib)
+    assert L.spkv_encode_keys_packed(ctypes.byref(c), P, None, P, -1, 4, P, P, 4, None) == 1
+    assert L.spkv_encode_keys_packed(ctypes.byref(c), P + 4, None, P, 1, 4, P, P, 4, None) == 1
+    assert L.spkv_encode_keys_packed(ctypes.byref(c), P, None, P, 1, 0, P, P, 4, None) == 0
