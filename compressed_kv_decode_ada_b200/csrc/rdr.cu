@@ -355,12 +355,10 @@ __global__ void __launch_bounds__(kRdrThreads, 1) rdr_plan_kernel(const PlanPara
     return d.need ? rdr_choose(wget(j), p, L.r, L.z) : d.i;
   };
 
-  // One pass at multiplier lam: this CTA's tokens are evaluated, the CTAs'
-  // counts are exchanged (each CTA stores its record into every CTA's
-  // part[buf]), and every thread sums the records in rank order.  Returns
-  // the buffer the records are in.
-  auto count_pass = [&](double lam, uint32_t (&tot)[kTiers], uint32_t &ptot) -> int {
-    const PassLam L = pass_lam(lam, p);
+  // One pass with the multiplier in L: this CTA's tokens are evaluated and
+  // the CTAs' counts are exchanged (each CTA stores its record into every
+  // CTA's part[buf]).  Returns the buffer the records are in.
+  auto count_pass = [&](const PassLam &L) -> int {
     uint32_t c[kTiers] = {0u, 0u, 0u, 0u}, np = 0u;
     // groups of 4 tokens per thread decided without branches; a warp-wide
     // vote sends the (rare) abstentions to fp64.  The trip count is the same
@@ -413,21 +411,24 @@ __global__ void __launch_bounds__(kRdrThreads, 1) rdr_plan_kernel(const PlanPara
       if (lane < kRdrCluster) *cluster.map_shared_rank(&part[buf][rank], lane) = rec;
     }
     cluster.sync();
+    const int used = buf;
+    buf ^= 1;
+    return used;
+  };
+  // Every CTA's counts of the pass whose records are in part[b], summed in rank order.
+  auto totals = [&](int b, uint32_t (&tot)[kTiers], uint32_t &ptot) {
 #pragma unroll
     for (int j = 0; j < kTiers; ++j) tot[j] = 0u;
     ptot = 0u;
 #pragma unroll
     for (int r = 0; r < kRdrCluster; ++r) {
-      const CtaCounts &q = part[buf][r];
+      const CtaCounts &q = part[b][r];
       tot[0] += q.n.x;
       tot[1] += q.n.y;
       tot[2] += q.n.z;
       tot[3] += q.n.w;
       ptot += q.prot;
     }
-    const int used = buf;
-    buf ^= 1;
-    return used;
   };
   auto rate_of = [&](const uint32_t (&tot)[kTiers]) -> double {
     uint64_t r = 0;
@@ -436,40 +437,92 @@ __global__ void __launch_bounds__(kRdrThreads, 1) rdr_plan_kernel(const PlanPara
     return (double)r;
   };
 
-  // ---- the multiplier (every thread takes the same steps)
-  uint32_t tot[kTiers], ptot;
-  double lam = 0.0;
-  int st = 0;
-  count_pass(0.0, tot, ptot);
-  if (rate_of(tot) > budget) {
-    const double prot_rate = (double)((uint64_t)ptot * p.rate_u[p.imax]);
-    if (prot_rate > budget) {
-      st = SPKV_RDR_INFEASIBLE;  // protected tokens at b_max, every other one evicted
-      lam = INFINITY;
-    } else {
-      double hi = 1.0;
-      for (int n = 0; n < kMaxDoublings; ++n) {
-        count_pass(hi, tot, ptot);
-        if (!(rate_of(tot) > budget)) break;
-        hi *= 2.0;
+  // ---- the multiplier.  Thread 0 of each CTA steps the search (the same
+  // records give every CTA the same steps), in the oracle's order: lambda = 0;
+  // if over budget and feasible, doubling from 1, then bisection on [lo, hi]
+  // until the midpoint equals an end of the bracket (rate(lo) > budget and
+  // rate(hi) <= budget throughout, so the remaining halvings would leave it
+  // unchanged) or 100 halvings.  It publishes the next multiplier (with its
+  // per-tier products) through shared memory: the scalar fp64 work is done
+  // once per CTA, not by every thread.
+  __shared__ PassLam ctl_L;
+  __shared__ int ctl_go;
+  double lam = 0.0, cur = 0.0, lo = 0.0, hi = 1.0;  // (thread 0)
+  int st = 0, phase = 0, n = 0, it = 0;             // (thread 0)
+  if (tid == 0) {
+    ctl_L = pass_lam(0.0, p);
+    ctl_go = 1;
+  }
+  __syncthreads();
+  while (ctl_go) {  // (read after a __syncthreads: the same on every thread)
+    const PassLam L = ctl_L;
+    const int b = count_pass(L);
+    if (tid == 0) {
+      uint32_t tot[kTiers], ptot;
+      totals(b, tot, ptot);
+      const bool over = rate_of(tot) > budget;
+      bool done = false, bisect = false;
+      double next = 0.0;
+      if (phase == 0) {  // lambda = 0
+        if (!over) {
+          done = true;
+          lam = 0.0;
+        } else if ((double)((uint64_t)ptot * p.rate_u[p.imax]) > budget) {
+          done = true;  // protected tokens at b_max, every other one evicted
+          st = SPKV_RDR_INFEASIBLE;
+          lam = INFINITY;
+        } else {
+          phase = 1;
+          hi = 1.0;
+          n = 0;
+          next = hi;
+        }
+      } else if (phase == 1) {  // doubling: cur = hi
+        if (!over) {
+          bisect = true;
+        } else {
+          hi *= 2.0;
+          ++n;
+          if (n < kMaxDoublings) next = hi;
+          else bisect = true;
+        }
+        if (bisect) {
+          phase = 2;
+          lo = 0.0;
+          it = 0;
+        }
+      } else {  // bisection: cur = the midpoint just evaluated
+        if (over) lo = cur;
+        else hi = cur;
+        ++it;
+        bisect = true;
       }
-      // rate(lo) > budget and rate(hi) <= budget throughout, so once the
-      // midpoint equals lo or hi no further halving changes the bracket
-      double lo = 0.0;
-      for (int it = 0; it < kBisections; ++it) {
+      if (bisect) {
         const double mid = __dmul_rn(0.5, __dadd_rn(lo, hi));
-        if (mid == lo || mid == hi) break;
-        count_pass(mid, tot, ptot);
-        if (rate_of(tot) > budget) lo = mid;
-        else hi = mid;
+        if (it >= kBisections || mid == lo || mid == hi) {
+          done = true;
+          lam = hi;
+        } else {
+          next = mid;
+        }
       }
-      lam = hi;
+      if (done) {
+        ctl_go = 0;
+        ctl_L = pass_lam(lam, p);
+      } else {
+        cur = next;
+        ctl_L = pass_lam(next, p);
+      }
     }
+    __syncthreads();
   }
 
   // ---- the plan at lam: counts (and every CTA's counts, for the packing)
-  const int fb = count_pass(lam, tot, ptot);
-  const double rate = rate_of(tot);
+  const PassLam Lf = ctl_L;
+  const int fb = count_pass(Lf);
+  uint32_t tot[kTiers], ptot;
+  totals(fb, tot, ptot);
+  const double rate = tid == 0 ? rate_of(tot) : 0.0;  // (reported by thread 0 of rank 0)
   int64_t pstart[kTiers], npg[kTiers], total_pages = 0;
 #pragma unroll
   for (int j = 0; j < kTiers; ++j) {
@@ -490,7 +543,6 @@ __global__ void __launch_bounds__(kRdrThreads, 1) rdr_plan_kernel(const PlanPara
   // ---- write sweep: tier, packed position (rank within the tier = tokens
   // of the tier before this one: earlier CTAs, earlier steps, earlier warps,
   // earlier lanes), and this CTA's share of the distortion
-  const PassLam Lf = pass_lam(lam, p);
   const uint32_t lt_mask = (1u << lane) - 1u;
   double dl = 0.0;
   int step = 0;
