@@ -30,7 +30,8 @@
 //   rdr_plan_kernel: one thread-block cluster of kRdrCluster CTAs per
 //     sequence; each pass evaluates every token at one lambda, the CTAs
 //     exchange their per-tier counts through distributed shared memory, and
-//     every thread takes the same bisection step.  The bisection stops once
+//     thread 0 of every CTA takes the same bisection step from the same
+//     counts and publishes the next lambda to its CTA.  The bisection stops once
 //     the midpoint equals an end of the bracket (the remaining halvings
 //     cannot move it).  The last pass writes the tiers and packs the
 //     resident tokens into pages: tiers ascending, tokens ascending within
