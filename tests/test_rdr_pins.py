@@ -152,3 +152,39 @@ def test_pack_makes_tier_homogeneous_pages(seed):
     assert len(bits) == sum(-(-int(np.sum(tiers == b)) // 16) for b in (3, 4, 6, 8))
     for b in (3, 4, 6, 8):  # ascending t within a tier
         assert np.all(np.diff(dst[tiers == b]) > 0)
+
+
+@pytest.mark.parametrize("seed", [10, 11])
+def test_packed_layout_gives_the_attention_of_the_kept_tokens(seed):
+    """Attention over the packed pages (tokens moved to dst_pos, page bit
+    widths, slot keep bits) equals attention over the kept tokens in their
+    original order with the plan's tiers: the packing loses, duplicates and
+    re-tiers nothing."""
+    rng = np.random.default_rng(seed)
+    T, H, d, G = 150, 2, 128, 2
+    keys = _keys(rng, T, H, d)
+    vals = _keys(rng, T, H, d, scale=1.0)
+    qn = rng.uniform(0.5, 2.0, H)
+    protect = np.zeros(T, np.uint8)
+    protect[:4] = 1
+    tiers, _, _, _, st = oracle.rdr_plan(keys, qn, 0.3 * T * _rate(8, H), protect=protect)
+    assert st == 0 and np.any(tiers == 0) and len(set(tiers[tiers > 0].tolist())) > 1
+    dst, pbits, pkeep = oracle.rdr_pack(tiers)
+    n_slots = 16 * len(pbits)
+    kept = np.nonzero(tiers > 0)[0]
+    for h in range(H):
+        q = _keys(rng, G, 1, d)[:, 0]
+        L, D = -2.0, 0.05
+        bits0 = np.where(tiers > 0, tiers, 8).astype(np.int32)
+        c0, r0 = oracle.encode(keys[:, h], bits0, L, D)
+        ref = oracle.ada_group(q, c0, bits0, r0, L, D, vals[:, h], keep=(tiers > 0).astype(np.uint8))
+        # the packed sequence: slot s of page p holds the token with dst = 16 p + s
+        pk = np.zeros((n_slots, d), np.uint16)
+        pv = np.zeros((n_slots, d), np.uint16)
+        pk[dst[kept]] = keys[kept, h]
+        pv[dst[kept]] = vals[kept, h]
+        sbits = np.repeat(pbits.astype(np.int32), 16)
+        skeep = ((pkeep[:, None].astype(np.int64) >> np.arange(16)) & 1).reshape(-1).astype(np.uint8)
+        c1, r1 = oracle.encode(pk, sbits, L, D)
+        got = oracle.ada_group(q, c1, sbits, r1, L, D, pv, keep=skeep)
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
