@@ -78,6 +78,8 @@ def lib():
         L.spkv_oracle_ada_group_exact_q.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _d, _d, _p, _p, _p, _p]
         L.spkv_oracle_rdr_plan.restype = _i
         L.spkv_oracle_rdr_plan.argtypes = [_i, _i, _i, _p, _p, _p, _d, ctypes.c_uint32, _p, _p, _p, _p]
+        L.spkv_oracle_rdr_assign.restype = _d
+        L.spkv_oracle_rdr_assign.argtypes = [_i, _i, _i, _p, _p, _p, ctypes.c_uint32, _d, _p]
         L.spkv_oracle_dense_group.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _p]
         _lib = L
     return _lib
@@ -267,6 +269,19 @@ def rdr_plan(keys_bf16, q_norms, budget_bytes, tier_mask=0xF, protect=None):
     st = lib().spkv_oracle_rdr_plan(d, T, Hkv, _ptr(k), _ptr(qn), _ptr(pr), float(budget_bytes), int(tier_mask),
                                     _ptr(tiers), ctypes.byref(lam), ctypes.byref(rate), ctypes.byref(dist))
     return tiers, lam.value, rate.value, dist.value, int(st)
+
+
+
+def rdr_assign(keys_bf16, q_norms, lam, tier_mask=0xF, protect=None):
+    """Tiers [T] and total rate of the per-token minimisers at one multiplier lam."""
+    k = _c(keys_bf16, np.uint16)
+    T, Hkv, d = k.shape
+    qn = _c(np.asarray(q_norms, np.float64).reshape(Hkv), np.float64)
+    pr = _c(protect, np.uint8)
+    tiers = np.empty(T, np.int32)
+    rate = lib().spkv_oracle_rdr_assign(d, T, Hkv, _ptr(k), _ptr(qn), _ptr(pr), int(tier_mask), float(lam),
+                                        _ptr(tiers))
+    return tiers, rate
 
 
 RDR_TIER_ORDER = (3, 4, 6, 8)

@@ -475,3 +475,30 @@ int spkv_oracle_rdr_plan(int d, int T, int Hkv, const uint16_t *keys, const doub
     free(w);
     return status;
 }
+
+/* The assignment at one multiplier (the step the bisection repeats): tiers of
+ * every token at lambda and their total rate, with the weights w_t as in
+ * spkv_oracle_rdr_plan.  Exposed for the pins of the solver. */
+double spkv_oracle_rdr_assign(int d, int T, int Hkv, const uint16_t *keys, const double *qn, const uint8_t *protect,
+                              uint32_t tier_mask, double lambda, int32_t *tier)
+{
+    int bmax = 0;
+    for (int i = 0; i < 4; ++i)
+        if ((tier_mask >> i) & 1u) bmax = kRdrBits[i];
+    double *w = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    for (int t = 0; t < T; ++t) {
+        double wt = 0.0;
+        for (int h = 0; h < Hkv; ++h) {
+            double n2 = 0.0;
+            for (int j = 0; j < d; ++j) {
+                const double x = spkv_oracle_bf16_to_f64(keys[((size_t)t * Hkv + h) * d + j]);
+                n2 += x * x;
+            }
+            wt += qn[h] * sqrt(n2);
+        }
+        w[t] = wt;
+    }
+    const double rate = rdr_assign(T, Hkv, w, protect, tier_mask, bmax, lambda, tier);
+    free(w);
+    return rate;
+}

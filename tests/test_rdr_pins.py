@@ -188,3 +188,25 @@ def test_packed_layout_gives_the_attention_of_the_kept_tokens(seed):
         c1, r1 = oracle.encode(pk, sbits, L, D)
         got = oracle.ada_group(q, c1, sbits, r1, L, D, pv, keep=skeep)
         np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("frac", [0.2, 0.45, 0.7])
+def test_multiplier_is_the_smallest_that_fits(frac):
+    """The solver's lambda fits the budget and the next smaller double does
+    not (the bisection converges to adjacent doubles); its tiers are the
+    per-token minimisers at lambda."""
+    rng = np.random.default_rng(12)
+    T, H, d = 300, 4, 64
+    keys = _keys(rng, T, H, d)
+    qn = rng.uniform(0.5, 2.0, H)
+    budget = frac * T * _rate(8, H)
+    tiers, lam, rate, _, st = oracle.rdr_plan(keys, qn, budget)
+    assert st == 0 and 0.0 < lam < math.inf
+    t_at, r_at = oracle.rdr_assign(keys, qn, lam)
+    np.testing.assert_array_equal(t_at, tiers)
+    assert r_at == rate <= budget
+    _, r_below = oracle.rdr_assign(keys, qn, np.nextafter(lam, 0.0))
+    assert r_below > budget
+    # rate is non-increasing in lambda
+    rates = [oracle.rdr_assign(keys, qn, x)[1] for x in np.geomspace(lam / 64, lam * 64, 25)]
+    assert all(a >= b for a, b in zip(rates, rates[1:]))
