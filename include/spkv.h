@@ -354,8 +354,10 @@ SPKV_API spkv_status spkv_debug_wait_timeout(uint32_t *err_flags, int32_t *statu
 #define SPKV_RDR_PAGES 0x2      /* the packed plan needs more than max_pages_out
                                    pages: n_pages says how many; dst_pos = -1
                                    and no page entries written */
-#define SPKV_RDR_BAD_RANGE 0x4  /* seq_start out of order or out of range:
-                                   nothing else written for the sequence */
+#define SPKV_RDR_BAD_RANGE 0x4  /* seq_start out of order or out of range: the
+                                   sequence's n_pages, lambda, rate and
+                                   distortion are 0; no tier, dst_pos or page
+                                   entry is written for it */
 
 SPKV_API size_t spkv_rdr_workspace_bytes(int64_t total_tokens);
 
