@@ -193,3 +193,13 @@ def test_plan_extreme_weights(spkv):
         ri = syn.make_rdr_inputs(wl, budget_frac=frac)
         _check(wl, ri, _plan(m, wl, ri))
         _check(wl, ri, _plan(m, wl, ri, protect=False), protect=False)
+
+
+def test_plan_sequence_longer_than_shared_memory(spkv):
+    """One sequence of 140,000 tokens: each CTA's share (17,500) exceeds the
+    16,384 weights it keeps in shared memory, so the rest is read from global
+    memory on every pass."""
+    m, syn = spkv
+    wl = syn.make_workload(RAGGED, B=1, ctx=[140000], Hq=1, Hkv=1, seed=26)
+    ri = syn.make_rdr_inputs(wl, budget_frac=0.4)
+    _check(wl, ri, _plan(m, wl, ri))
