@@ -272,9 +272,12 @@ def rdr_plan(keys: torch.Tensor, seq_start: torch.Tensor, q_norms: torch.Tensor,
              ws: torch.Tensor | None = None, stream=None) -> dict:
     """spkv_rdr_plan over sequences concatenated in keys [total_tokens, H_kv, 128] bf16.
 
-    Returns a dict of device tensors: tier [T] uint8, dst_pos [T] int32,
-    page_bits / page_keep [B, max_pages_out], n_pages [B] int32, lambda,
-    rate, dist [B] float64, status [B] int32."""
+    Returns a dict of device tensors: tier [T] uint8 (b, 0 = evicted),
+    dst_pos [T] int32 (-1 = evicted), page_bits [B, max_pages_out] uint8,
+    page_keep [B, max_pages_out] int16 (the uint16 slot masks' bits),
+    n_pages [B] int32, lambda, rate, dist [B] float64, status [B] int32
+    (SPKV_RDR_* bits).  max_pages_out defaults to ceil(T / 16) + 3, enough
+    for any sequence of the batch."""
     _need(keys, torch.bfloat16, "keys", 3)
     total, hkv, d = keys.shape
     if d != HEAD_DIM:
