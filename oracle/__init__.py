@@ -9,8 +9,11 @@ The arithmetic lives in ``spkv_oracle.c`` (plain C, IEEE fp64); this module
 only builds it with gcc and marshals numpy arrays through ctypes.  Each wrapper
 cites the definition it follows: "SPHERICAL KV: Angle-Domain Attention and
 Rate-Distortion Retention for Efficient Long-Context Inference", technical
-summary section 2.1 (Angle-Domain Attention).  The readings R1-R7 where the
-pages are silent are listed at the top of ``spkv_oracle.c``.
+summary section 2.1 (Angle-Domain Attention) and section 2.2 (Rate-Distortion
+Retention: ``rdr_plan``, ``rdr_assign``, ``rdr_pack``).  The readings where the
+pages are silent are listed at the top of ``spkv_oracle.c`` (R1-R13) and at
+the RDR controller in it (R14-R17); ``rdr_pack`` states R18 and
+``nonuniform.py`` (the non-uniform angle quantiser) R19.
 
 ctypes drops the GIL around each foreign call, so ``map_groups`` runs the
 per-(sequence, kv head) oracle calls on a thread pool.
