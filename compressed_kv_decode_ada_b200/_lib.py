@@ -37,6 +37,7 @@ EXPORTS = (
     "spkv_rdr_workspace_bytes",
     "spkv_rdr_plan",
     "spkv_encode_keys_packed",
+    "spkv_nonuniform_tables",
 )
 PARTIAL_FLOATS = 132  # floats per (sequence, query head) shard record
 DECODE_EXACT_Q = 1  # SPKV_DECODE_EXACT_Q
@@ -126,6 +127,8 @@ def _load():
     L.spkv_encode_keys_packed.restype = ctypes.c_int
     L.spkv_encode_keys_packed.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _P, _P, _I, ctypes.c_int64, _P, _P, _I,
                                           _P]
+    L.spkv_nonuniform_tables.restype = ctypes.c_int
+    L.spkv_nonuniform_tables.argtypes = [_I, _I, _P, _P, _P]
     return L
 
 

@@ -310,3 +310,16 @@ def rdr_plan(keys: torch.Tensor, seq_start: torch.Tensor, q_norms: torch.Tensor,
                             _ptr(out["n_pages"]), _ptr(out["lambda"]), _ptr(out["rate"]), _ptr(out["dist"]),
                             _ptr(out["status"]), _ptr(ws), ws.numel(), _stream(stream)), "spkv_rdr_plan")
     return out
+
+
+def nonuniform_tables(d: int, b: int):
+    """spkv_nonuniform_tables: (edge_cos [d-2, 2^b-1], mid_cos [d-2, 2^b],
+    mid_sin [d-2, 2^b]) as fp64 numpy arrays (host computation)."""
+    import numpy as np
+
+    n = 1 << b
+    ec = np.empty((max(d - 2, 1), n - 1), np.float64)
+    mc = np.empty((max(d - 2, 1), n), np.float64)
+    ms = np.empty((max(d - 2, 1), n), np.float64)
+    check(lib.spkv_nonuniform_tables(d, b, ec.ctypes.data, mc.ctypes.data, ms.ctypes.data), "spkv_nonuniform_tables")
+    return ec[:d - 2], mc[:d - 2], ms[:d - 2]

@@ -383,6 +383,20 @@ SPKV_API spkv_status spkv_encode_keys_packed(const spkv_cache *cache, const uint
                                              const int32_t *dst_pos, const int32_t *block_table, int32_t max_pages,
                                              void *stream);
 
+/* Host tables of the non-uniform angle quantiser (an f_b variant; technical
+ * summary section 2.1 leaves the quantiser open).  Reading: for a direction
+ * drawn uniformly on the unit sphere of R^d, polar angle phi_i (i = 1..d-2)
+ * has the density sin^(d-1-i)(phi)/Z on [0, pi]; each polar angle gets 2^b
+ * cells of equal probability (edges at the j/2^b quantiles) reconstructed at
+ * the cell median (the (j+1/2)/2^b quantile); the azimuth keeps the uniform
+ * cells.  Computed on the host in fp64 (no GPU, no stream):
+ *   edge_cos [(d-2) * (2^b - 1)]  cos of edge j = 1..2^b-1 of angle i, row i-1
+ *   mid_cos, mid_sin [(d-2) * 2^b] cos / sin of the reconstruction angles
+ * All three are caller-owned host arrays.  d in 3..4096, b in 1..12, else
+ * SPKV_ERR_INVALID_ARG with nothing written. */
+SPKV_API spkv_status spkv_nonuniform_tables(int32_t d, int32_t b, double *edge_cos, double *mid_cos,
+                                            double *mid_sin);
+
 #ifdef __cplusplus
 }
 #endif
