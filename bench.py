@@ -55,6 +55,23 @@ def _dist():
     return rank, world, local
 
 
+def _synthetic_inputs():
+    """The seeded input generators (compressed_kv_decode_ada_b200/synthetic.py),
+    loaded from their file without importing the package: the package's
+    __init__ maps libspkv.so, which the CPU oracle arm must not load."""
+    import importlib.util
+
+    name = "_spkv_synthetic_inputs"
+    if name in sys.modules:
+        return sys.modules[name]
+    path = os.path.join(ROOT, "compressed_kv_decode_ada_b200", "synthetic.py")
+    spec = importlib.util.spec_from_file_location(name, path)
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[name] = mod
+    spec.loader.exec_module(mod)
+    return mod
+
+
 def _cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -396,8 +413,8 @@ def cpu_oracle(args, budget_s: float):
     import torch
 
     import oracle
-    from compressed_kv_decode_ada_b200 import synthetic
 
+    synthetic = _synthetic_inputs()
     cfg = dict(synthetic.WORKLOADS[args.workload])
     wl = synthetic.make_workload(cfg, device="cpu", B=min(cfg["B"], 2))
     cores = _cores()
@@ -495,8 +512,6 @@ def main():
         if rank != 0:
             return 0
         cb = cpu_oracle(args, args.cpu_budget)
-        from compressed_kv_decode_ada_b200 import synthetic
-
         line = {"metric": "ADA decode KV tokens/s on 1 B200; achieved HBM GB/s as % of peak", "impl": "reference",
                 "value": cb["value"], "unit": "KV tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",

@@ -68,3 +68,21 @@ def test_single_process_needs_no_collective():
 
     assert bench.max_over_ranks([3.0, 1.0]) == [3.0, 1.0]
     assert bench.whole_job_rate(10.0, 1, 1.0) == pytest.approx(1e4)
+
+
+def test_reference_arm_maps_only_the_oracle_library():
+    """bench.py --impl reference times the oracle alone: the process that runs
+    it loads the input generators but neither the package nor libspkv.so."""
+    import subprocess
+    import sys
+
+    code = (
+        "import sys, types, bench\n"
+        "args = types.SimpleNamespace(workload='llama3_8b_b8_h32x8_t32768_b4')\n"
+        "cb = bench.cpu_oracle(args, 0.01)\n"
+        "maps = open('/proc/self/maps').read()\n"
+        "print(cb['kind'], cb['value'] > 0, 'compressed_kv_decode_ada_b200' in sys.modules,\n"
+        "      'libspkv.so' in maps, 'libspkv_oracle.so' in maps)\n")
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.split() == ["oracle", "True", "False", "False", "True"]
