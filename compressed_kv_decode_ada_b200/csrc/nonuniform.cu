@@ -16,6 +16,7 @@
 // by Newton's method on its three-term recurrence); a quantile is found by
 // locating its panel in the table, then Newton steps on
 // F_k(theta) - p = 0 with F_k' = sin^k / Z_k, kept inside the panel.
+#include <cfloat>
 #include <cmath>
 #include <vector>
 
@@ -108,11 +109,12 @@ struct SinePowerLaw {
       const double dens = sin_pow(t, k) / Z;
       double tn = dens > 0 ? t - f / dens : 0.5 * (a + b);
       if (!(tn > a && tn < b)) tn = 0.5 * (a + b);  // stay in the bracket
-      if (std::fabs(tn - t) <= 1e-17 * (1.0 + std::fabs(t))) {
-        t = tn;
-        break;
-      }
+      // done when the Newton step or the bracket is down to two ulps of t
+      // (the iteration cap is only a backstop)
+      const double two_ulps = 2.0 * DBL_EPSILON * std::fabs(t) + 1e-300;
+      const bool done = std::fabs(tn - t) <= two_ulps || b - a <= two_ulps;
       t = tn;
+      if (done) break;
     }
     return t;
   }

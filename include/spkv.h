@@ -263,14 +263,21 @@ SPKV_API spkv_status spkv_decompress_then_dot(const spkv_cache *cache, uint16_t 
  * split-partials workspace taken from an array of SPKV_STATIC_WS_BYTES that
  * the library holds in device memory on every device that loads it, until
  * the process exits; it allocates nothing itself.
- *   Arguments and results: as spkv_decode_attention, without ws / ws_bytes.
- *   Limit: returns SPKV_ERR_WORKSPACE when spkv_decode_workspace_bytes(B,
+ *   Arguments and results: as spkv_decode_attention, without ws / ws_bytes;
+ *   its argument checks run first, so an invalid argument gets the status it
+ *   gets there.
+ *   Limit: then returns SPKV_ERR_WORKSPACE when spkv_decode_workspace_bytes(B,
  *   num_q_heads, H_kv, max_ctx, num_splits) exceeds SPKV_STATIC_WS_BYTES
  *   (e.g. B = 8, 32 query / 8 kv heads and the default split count need
  *   about 4.6 MB).
- *   Set-up: the first call on a device, with that device current, looks up
- *   the array's device address (cudaGetSymbolAddress) and caches it; make
- *   that first call before any stream capture.
+ *   Set-up: the first call in a CUDA context, with the device current, looks
+ *   up the array's device address (cudaGetSymbolAddress) and caches it with
+ *   the context's id (cuCtxGetId); make that first call before any stream
+ *   capture.  A call from another context of the device -- after
+ *   cudaDeviceReset, or once the primary context was released and created
+ *   again, when the module is loaded at a new address -- looks the address up
+ *   again, so that first call in the new context must also come before any
+ *   capture.
  *   Sharing: every call on a device uses the same array, and each call
  *   overwrites what the previous one left there (nothing in it needs to start
  *   at zero).  Calls whose kernels overlap on the GPU (different streams, no

@@ -58,26 +58,7 @@ def _decode(spkv, wl, cache, **kw):
 # ------------------------------------------------------------------ encode
 
 def _check_codes(wl, cache, groups):
-    arena = cache.arena.cpu().numpy()
-    n_codes = n_edge = n_mismatch_edge = 0
-    for b, h in groups:
-        gc, gr, pads = helpers.gpu_codes_for_seq(arena, wl, b, h)
-        keys, bits = wl.keys_bits(b, h), wl.token_bits(b)
-        oc, orc, apos, rpos = oracle.encode(keys, bits, float(wl.rad_lo[h]), float(wl.rad_step[h]), positions=True)
-        edge_a, edge_r = helpers.near_integer(apos), helpers.near_integer(rpos)
-        bad_a = (gc != oc) & ~edge_a
-        bad_r = (gr != orc) & ~edge_r
-        assert not bad_a.any(), f"angle code mismatch off a cell edge at (b={b}, h={h}): {np.argwhere(bad_a)[:5]}"
-        assert not bad_r.any(), f"radius code mismatch off a cell edge at (b={b}, h={h})"
-        assert np.all(pads == 0)
-        n_codes += oc.size + orc.size
-        n_edge += int(edge_a.sum() + edge_r.sum())
-        n_mismatch_edge += int(((gc != oc) & edge_a).sum() + ((gr != orc) & edge_r).sum())
-    # codes decided differently on a cell edge (fp64 rounding either way) must
-    # stay below 1e-6 of all codes; exact ties (common with bf16 inputs, e.g.
-    # |x_126| = |x_127|) are decided exactly by both sides and counted as matches
-    assert n_mismatch_edge <= max(1, 1e-6 * n_codes), (n_mismatch_edge, n_edge, n_codes)
-    return n_codes, n_edge, n_mismatch_edge
+    return helpers.check_codes(wl, cache, groups)
 
 
 def test_encode_codes_bit_exact_tiny(spkv):

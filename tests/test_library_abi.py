@@ -83,6 +83,42 @@ def test_host_argument_checks(lib):
     assert L.spkv_encode_keys(ctypes.byref(c), 0x1000, None, 0x2000, 0, 1, 0x3000, 4, None) == 0
 
 
+def _static(m, c, B=1, Hq=4, splits=4, q=0x60000, max_ctx=128):
+    cp = ctypes.byref(c) if c is not None else None
+    return m.lib.spkv_decode_attention_static_ws(cp, q, B, Hq, 0x70000, 8, 0x80000, max_ctx, 0x90000, 0, splits, None)
+
+
+def test_static_ws_argument_checks_match_decode(lib):
+    """spkv_decode_attention_static_ws runs spkv_decode_attention's argument checks
+    before its own capacity check: a bad argument gets the same status from both
+    entry points, also when its workspace would exceed the fixed array."""
+    m = lib
+    L = m.lib
+
+    def dec(c, B=1, Hq=4, splits=4, q=0x60000, max_ctx=128):
+        cp = ctypes.byref(c) if c is not None else None
+        return L.spkv_decode_attention(cp, q, B, Hq, 0x70000, 8, 0x80000, max_ctx, 0x90000, 0, 0xA0000, 1 << 20,
+                                       splits, None)
+
+    cases = [
+        (None, {}),                                   # no cache
+        (_fake_cache(m, head_dim=64), {}),             # unsupported head dim
+        (_fake_cache(m), dict(Hq=6)),                  # G = 3
+        (_fake_cache(m), dict(Hq=3)),                  # Hq not a multiple of H_kv
+        (_fake_cache(m), dict(q=0x60002)),             # misaligned q
+        (_fake_cache(m), dict(B=5000, splits=4096)),   # batch beyond the maximum, workspace far beyond 16 MiB
+        (_fake_cache(m), dict(B=1024, max_ctx=1 << 24, splits=4096)),  # too many pages, huge workspace
+        (_fake_cache(m), dict(B=0)),                   # empty batch
+        (_fake_cache(m), dict(B=1024, splits=4096)),   # valid, but 39 MB of workspace: both too small
+    ]
+    want = [1, 2, 2, 1, 1, 2, 2, 0, 3]
+    for (c, kw), w in zip(cases, want):
+        assert dec(c, **kw) == w, kw
+        assert _static(m, c, **kw) == w, kw
+    need = m.workspace_bytes(1024, 4, 2, 128, 4096)
+    assert need > m._lib.STATIC_WS_BYTES
+
+
 def test_workspace_formula(lib):
     # (C + B H_kv) segments x 6 consumer-warp slots x G partials of 132 floats
     # (rounded to 16 bytes), then one 4-byte row counter per kv row (rounded)

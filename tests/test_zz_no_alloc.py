@@ -11,7 +11,6 @@ import torch
 
 pytestmark = pytest.mark.gpu
 
-OUT_TOL = 2e-3
 
 
 @pytest.fixture(scope="module")
@@ -49,7 +48,8 @@ def test_static_workspace_matches_allocated_workspace(spkv):
         torch.cuda.synchronize()
         assert st == 0, m.lib.spkv_status_string(st)
         assert cache.error_flags() == 0
-        assert torch.max(torch.abs(out - ref)).item() <= OUT_TOL
+        # the same kernels at the same split count: bit-identical output
+        assert torch.equal(out, ref)
 
 
 def test_static_workspace_rejects_sizes_beyond_its_capacity(spkv):
@@ -64,4 +64,33 @@ def test_static_workspace_rejects_sizes_beyond_its_capacity(spkv):
     ctx = torch.zeros(1024, dtype=torch.int32, device="cuda")
     out = torch.empty((1024, 32, 128), dtype=torch.float32, device="cuda")
     st = _static_ws_call(m, cache, q, bt, ctx, 1 << 20, out, num_splits=4096)
+    assert st == 3  # SPKV_ERR_WORKSPACE
+
+
+def test_static_workspace_capacity_boundary(spkv):
+    """An explicit split count whose workspace just fits the fixed array runs and
+    equals the caller-workspace call bit for bit; one more split is rejected."""
+    m, synthetic, workload = spkv
+    wl = synthetic.make_workload("llama3_8b_b8_h32x8_t32768_b4", device="cuda", B=8,
+                                 ctx=[64, 300, 17, 1000, 16, 512, 129, 2048])
+    cache = workload.build_cache(wl)
+    ctx = wl.ctx_tensor()
+    cap = m._lib.STATIC_WS_BYTES
+    lo, hi = 1, 1 << 16  # largest C whose workspace fits
+    while lo < hi:
+        mid = (lo + hi + 1) // 2
+        if m.workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.max_ctx, mid) <= cap:
+            lo = mid
+        else:
+            hi = mid - 1
+    c_max = lo
+    assert m.workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.max_ctx, c_max + 1) > cap
+    ref = m.decode_attention(cache, wl.q, wl.block_table, ctx, wl.max_ctx, num_splits=c_max)
+    out = torch.empty_like(ref)
+    st = _static_ws_call(m, cache, wl.q, wl.block_table, ctx, wl.max_ctx, out, num_splits=c_max)
+    torch.cuda.synchronize()
+    assert st == 0, m.lib.spkv_status_string(st)
+    assert cache.error_flags() == 0
+    assert torch.equal(out, ref)
+    st = _static_ws_call(m, cache, wl.q, wl.block_table, ctx, wl.max_ctx, out, num_splits=c_max + 1)
     assert st == 3  # SPKV_ERR_WORKSPACE
