@@ -486,6 +486,58 @@ def run_rdr(args):
             "status": plan["status"].cpu().tolist()[:8], "gpu_launches": 2 * args.steps}
 
 
+def run_profile_only(args):
+    """One path alone, for profiler captures: W warm-up and K calls of
+    'ada' (spkv_decode_attention), 'dense' (spkv_dense_decode), 'dtd'
+    (spkv_decompress_then_dot) or 'encode' (spkv_encode_keys of every context
+    key and value) on the workload, so a capture can skip and count its
+    launches exactly.  Prints one JSON line with the mean CUDA-event time."""
+    import torch
+
+    from compressed_kv_decode_ada_b200 import synthetic, workload
+    import compressed_kv_decode_ada_b200 as spkv
+
+    dev = torch.device("cuda", 0)
+    kw = {"B": args.B} if args.B else {}
+    wl = synthetic.make_workload(args.workload, device=dev, **kw)
+    cache = workload.build_cache(wl)
+    ctx = wl.ctx_tensor()
+    max_ctx = wl.max_ctx
+    stream = torch.cuda.current_stream(dev)
+    ws = spkv.alloc_workspace(wl.B, wl.Hq, wl.Hkv, max_ctx, args.splits, device=dev)
+    path = args.profile_only
+    if path == "ada":
+        fn = lambda: spkv.decode_attention(cache, wl.q, wl.block_table, ctx, max_ctx, ws=ws, num_splits=args.splits,
+                                           stream=stream)
+        per_call = ["split_kernel (ADA)", "merge_kernel"]
+    elif path == "dense":
+        kp, vp = workload.dense_pages(wl)
+        fn = lambda: spkv.dense_decode(kp, vp, wl.q, wl.block_table, ctx, max_ctx, ws=ws, num_splits=args.splits,
+                                       stream=stream)
+        per_call = ["split_kernel (dense)", "merge_kernel"]
+    elif path == "dtd":
+        ks = torch.empty_like(cache.v_pages)
+        fn = lambda: spkv.decompress_then_dot(cache, ks, wl.q, wl.block_table, ctx, max_ctx, ws=ws,
+                                              num_splits=args.splits, stream=stream)
+        per_call = ["decompress_kernel", "split_kernel (dense)", "merge_kernel"]
+    else:
+        fn = lambda: workload.prefill(cache, wl)
+        per_call = ["encode_kernel"]
+    torch.cuda.synchronize(dev)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    return {"profile_only": path, "workload": wl.name, "B": wl.B, "ms_per_call": ms, "calls": args.warmup + args.steps,
+            "launches_per_call": per_call, "kv_tokens": wl.kv_tokens, "err_flags": cache.error_flags()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -501,6 +553,8 @@ def main():
     ap.add_argument("--compare-steps", type=int, default=50)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-only", choices=["ada", "dense", "dtd", "encode"], default=None,
+                    help="run one path alone, --warmup + --steps calls (one JSON line; profiler captures)")
     ap.add_argument("--rdr", action="store_true",
                     help="time only spkv_rdr_plan on the workload's keys (one JSON line; profiler captures)")
     args = ap.parse_args()
@@ -525,6 +579,11 @@ def main():
     if args.rdr:
         if rank == 0:
             print(json.dumps(run_rdr(args)), flush=True)
+        return 0
+
+    if args.profile_only:
+        if rank == 0:
+            print(json.dumps(run_profile_only(args)), flush=True)
         return 0
 
     res = run_spkv(args, rank, world, local)

@@ -53,15 +53,17 @@ def shard_batch(block_table: np.ndarray, ctx: np.ndarray, world: int, rank: int)
 
 
 def gather_partials(partial: torch.Tensor, group=None) -> torch.Tensor:
-    """All ranks' records [R, B, Hq, 132] in rank order (all_gather_into_tensor)."""
+    """All ranks' records [R, B, Hq, 132] in rank order, on partial's device
+    (all_gather_into_tensor; a gloo group exchanges host copies)."""
     import torch.distributed as dist
 
     world = dist.get_world_size(group)
     partial = partial.contiguous()
-    if dist.get_backend(group) == "gloo":  # (host-side process groups)
-        parts = [torch.empty_like(partial) for _ in range(world)]
-        dist.all_gather(parts, partial, group=group)
-        return torch.stack(parts)
+    if dist.get_backend(group) == "gloo":  # host-side process groups: stage through host memory
+        host = partial.cpu()
+        parts = [torch.empty_like(host) for _ in range(world)]
+        dist.all_gather(parts, host, group=group)
+        return torch.stack(parts).to(partial.device)
     out = torch.empty((world,) + tuple(partial.shape), dtype=partial.dtype, device=partial.device)
     dist.all_gather_into_tensor(out, partial, group=group)
     return out

@@ -189,3 +189,67 @@ def test_gpu_page_shards_merge_to_the_one_shot_decode(shards):
     assert torch.max(torch.abs(out - full)).item() <= _reorder_tol(wl)
     err = helpers.max_abs_diff_groups(out.cpu().numpy(), wl, helpers.all_groups(wl), helpers.oracle_seq)
     assert err <= 2e-3, err
+
+
+def _gpu_rank_main(rank, world, port, q):
+    """One rank of the composed sharded_decode on the one GPU: the CUDA partial
+    over this rank's pages, the gloo all-gather (host-staged), the CUDA merge."""
+    import datetime
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        from compressed_kv_decode_ada_b200 import synthetic, workload
+        from compressed_kv_decode_ada_b200.sharded import shard_batch, sharded_decode
+
+        wl = synthetic.make_workload(*_SHARD_WL, device="cuda", **_SHARD_KW)
+        cache = workload.build_cache(wl)
+        lbt, lctx = shard_batch(wl.block_table.cpu().numpy(), wl.ctx, world, rank)
+        out = sharded_decode(cache, wl.q, torch.from_numpy(lbt).cuda(), torch.from_numpy(lctx).cuda(),
+                             int(lctx.max()))
+        torch.cuda.synchronize()
+        q.put((rank, out.cpu().numpy(), cache.error_flags()))
+    finally:
+        dist.destroy_process_group()
+
+
+_SHARD_WL = ("ragged_rdr_b32_h32x8_t1k-64k_mixed_b_mask25",)
+_SHARD_KW = dict(B=3, ctx=[5000, 33, 2049], Hq=8, Hkv=2)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("world", [2, 3])
+def test_gpu_gloo_ranks_sharded_decode_end_to_end(world):
+    """sharded_decode as one function on every rank (gloo ranks sharing the GPU;
+    no kernel waits on another rank): every rank's output is the whole-sequence
+    attention of the oracle and the one-shot decode."""
+    import torch.multiprocessing as mp
+
+    import compressed_kv_decode_ada_b200 as m
+    from compressed_kv_decode_ada_b200 import synthetic, workload
+
+    from tests import helpers
+
+    port = _free_port()
+    ctxm = mp.get_context("spawn")
+    qu = ctxm.Queue()
+    procs = [ctxm.Process(target=_gpu_rank_main, args=(r, world, port, qu)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted((qu.get(timeout=300) for _ in range(world)), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    wl = synthetic.make_workload(*_SHARD_WL, device="cuda", **_SHARD_KW)
+    cache = workload.build_cache(wl)
+    full = m.decode_attention(cache, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx).cpu().numpy()
+    for rank, out, err_flags in res:
+        assert err_flags == 0
+        assert np.max(np.abs(out - full)) <= _reorder_tol(wl)
+        assert np.array_equal(out, res[0][1])  # every rank merged the same records
+    err = helpers.max_abs_diff_groups(res[0][1], wl, helpers.all_groups(wl), helpers.oracle_seq)
+    assert err <= 2e-3, err
