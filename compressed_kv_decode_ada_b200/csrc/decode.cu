@@ -678,12 +678,12 @@ constexpr int kPartial = 132;
 // new value row goes to the same slot of the value page.  Called before the
 // page's copy is issued; the caller fences the stores for the async proxy.
 __device__ __noinline__ void append_token(const SplitParams &p, int b, int h, int pid, int bits, uint64_t rec_off,
-                                          const double *pol_c2, const double *az_c2, uint8_t *codes_smem,
-                                          int lane) {
+                                          const double *pol_c2, const double *az_c2, int lane) {
   const int slot = (p.ctx_lens[b] - 1) % kPage;
   const int64_t row = (int64_t)b * p.Hkv + h;
-  encode_key_warp(p.new_k + row * kD, bits, const_cast<uint8_t *>(p.arena) + rec_off, slot, p.rad_lo[h],
-                  p.rad_step[h], pol_c2, az_c2, codes_smem, lane, p.err);
+  // the key: the warp form of spkv_encode_keys' arithmetic (the same bytes)
+  encode_key_warp_seq_bits(bits, p.new_k + row * kD, const_cast<uint8_t *>(p.arena) + rec_off, slot, p.rad_lo[h],
+                           p.rad_step[h], pol_c2, az_c2, lane, p.err);
   const uint2 v = *reinterpret_cast<const uint2 *>(p.new_v + row * kD + 4 * lane);
   *reinterpret_cast<uint2 *>(const_cast<uint16_t *>(p.v_pages) + (((int64_t)pid * p.Hkv + h) * kPage + slot) * kD +
                              4 * lane) = v;
@@ -706,7 +706,6 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
   // built once per CTA
   double *pol_c2 = reinterpret_cast<double *>(smem + Ly::off_pe);
   double *az_c2 = pol_c2 + kLutEntries;
-  uint8_t *pe_codes = smem + Ly::off_pe + 2 * kLutEntries * 8;
   float *pbuf_all = reinterpret_cast<float *>(smem + Ly::off_pbuf);
   float *sc = reinterpret_cast<float *>(smem + Ly::off_sc);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + Ly::off_bar);
@@ -835,7 +834,7 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
             todo &= todo - 1;
             append_token(p, __shfl_sync(0xffffffffu, ac.b, src), __shfl_sync(0xffffffffu, ac.h, src),
                          __shfl_sync(0xffffffffu, ac.pid, src), __shfl_sync(0xffffffffu, bc.bits, src),
-                         __shfl_sync(0xffffffffu, x.rec_off, src), pol_c2, az_c2, pe_codes, lane);
+                         __shfl_sync(0xffffffffu, x.rec_off, src), pol_c2, az_c2, lane);
           }
           // the copies below (and the consumers' value TMA) read what was written
           __threadfence();
@@ -952,7 +951,7 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
                 todo &= todo - 1;
                 append_token(p, __shfl_sync(0xffffffffu, ac.b, src), __shfl_sync(0xffffffffu, ac.h, src),
                              __shfl_sync(0xffffffffu, ac.pid, src), __shfl_sync(0xffffffffu, bc.bits, src),
-                             __shfl_sync(0xffffffffu, rec_off, src), pol_c2, az_c2, pe_codes, lane);
+                             __shfl_sync(0xffffffffu, rec_off, src), pol_c2, az_c2, lane);
               }
               // the copies below (and the consumers' value TMA) read what was written
               __threadfence();

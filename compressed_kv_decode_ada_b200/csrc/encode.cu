@@ -12,17 +12,17 @@
 //   phi_i >= theta_k  <=>  x_i <= sqrt(S_i) cos(theta_k)
 // (S_i = sum_{j >= i} x_j^2) is decided from x_i^2 versus S_i cos^2(theta_k)
 // plus the signs.  The code is the largest k whose edge theta_k the angle
-// reaches (binary search over the 2^b - 1 edges), i.e. floor(phi 2^b / pi)
-// clamped to 2^b - 1 -- ties go to the upper cell.  The azimuth (angle 127,
-// range [0, 2 pi)) uses the same test on (x_126, x_127) with the half-plane
-// given by the sign of x_127.  The radius code uses fp64 log2.
+// reaches (a binary search over the edges of the half of [0, pi] the sign of
+// x_i gives), i.e. floor(phi 2^b / pi) clamped to 2^b - 1 -- ties go to the
+// upper cell.  The azimuth (angle 127, range [0, 2 pi)) uses the same test on
+// (x_126, x_127) with the half-plane given by the sign of x_127.  The radius
+// code uses fp64 log2.  One thread encodes one key (spkv_encode.cuh).
 #include "spkv_encode.cuh"
 
 namespace spkv {
 namespace {
 
 constexpr int kEncThreads = 256;
-constexpr int kEncWarps = kEncThreads / 32;
 
 struct EncodeParams {
   uint8_t *arena;
@@ -42,69 +42,99 @@ struct EncodeParams {
 struct EncodeSmem {
   double pol_c2[kLutEntries];
   double az_c2[kLutEntries];
-  uint8_t codes[kEncWarps][128];
 };
 
-__global__ void __launch_bounds__(kEncThreads) encode_kernel(const EncodeParams p) {
+// Where item (key, kv head) `item` goes: its kv head, page and slot, or the
+// device-error bits that rule it out; skip: a packed token with a negative
+// position (nothing to write).
+struct EncPlace {
+  int h, pid, slot;
+  uint32_t st;
+  bool skip;
+};
+
+__device__ __forceinline__ EncPlace enc_place(const EncodeParams &p, int64_t item) {
+  EncPlace pl{0, -1, 0, 0u, false};
+  int64_t bn;
+  if (p.items <= 0x7fffffff) {  // 32-bit division where it fits
+    const uint32_t i32 = (uint32_t)item, hk = (uint32_t)p.Hkv, q = i32 / hk;
+    pl.h = (int)(i32 - q * hk);
+    bn = q;
+  } else {
+    pl.h = (int)(item % p.Hkv);
+    bn = item / p.Hkv;
+  }
+  int b, pos;
+  if (p.dst_pos) {  // token bn of the concatenated sequences, to dst_pos[bn]
+    pos = p.dst_pos[bn];
+    if (pos < 0) {
+      pl.skip = true;
+      return pl;
+    }
+    int lo = 0, hi = p.B;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if ((int64_t)p.seq_start[mid] <= bn) lo = mid;
+      else hi = mid;
+    }
+    b = lo;
+    if (bn < (int64_t)p.seq_start[b] || bn >= (int64_t)p.seq_start[b + 1]) {
+      pl.st = SPKV_DEVERR_CTX;
+      return pl;
+    }
+  } else if (bn <= 0xffffffffLL) {
+    const uint32_t nn = (uint32_t)p.n_new, q = (uint32_t)bn / nn;
+    b = (int)q;
+    pos = p.start_pos[b] + (int)((uint32_t)bn - q * nn);
+  } else {
+    b = (int)(bn / p.n_new);
+    pos = p.start_pos[b] + (int)(bn % p.n_new);
+  }
+  if (pos < 0 || pos >= p.max_pages * kPage) {
+    pl.st = SPKV_DEVERR_CTX;
+    return pl;
+  }
+  pl.slot = pos % kPage;
+  pl.pid = p.block_table[(int64_t)b * p.max_pages + pos / kPage];
+  if (pl.pid < 0 || pl.pid >= p.num_pages) pl.st = SPKV_DEVERR_PAGE_ID;
+  return pl;
+}
+
+// One thread per item: its placement, its page header, the key's codes
+// (encode_key_lane) and its value row.
+__global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const EncodeParams p) {
   __shared__ EncodeSmem sm;
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  build_edge_tables(sm.pol_c2, sm.az_c2, tid, kEncThreads);
+  build_edge_tables(sm.pol_c2, sm.az_c2, threadIdx.x, kEncThreads);
   __syncthreads();
-
-  const int64_t nwarps = (int64_t)gridDim.x * kEncWarps;
-  for (int64_t item = (int64_t)blockIdx.x * kEncWarps + wid; item < p.items; item += nwarps) {
-    const int h = (int)(item % p.Hkv);
-    const int64_t bn = item / p.Hkv;
-    int b, pos;
-    if (p.dst_pos) {  // token bn of the concatenated sequences, to dst_pos[bn]
-      pos = p.dst_pos[bn];
-      if (pos < 0) continue;
-      int lo = 0, hi = p.B;
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if ((int64_t)p.seq_start[mid] <= bn) lo = mid;
-        else hi = mid;
+  const int64_t step = (int64_t)gridDim.x * kEncThreads;
+  for (int64_t item = (int64_t)blockIdx.x * kEncThreads + threadIdx.x; item < p.items; item += step) {
+    const EncPlace pl = enc_place(p, item);
+    if (pl.skip) continue;
+    uint32_t st = pl.st;
+    int bits = 0;
+    uint64_t rec = 0;
+    if (!st) {
+      const spkv_page_hdr hd = p.hdr[pl.pid];
+      bits = hd.bits;
+      if (tier_of_bits(bits) < 0) {
+        st = SPKV_DEVERR_BITS;
+      } else {
+        rec = (uint64_t)hd.code_off16 * 16u + (uint64_t)pl.h * rec_bytes(bits);
+        if (rec + rec_bytes(bits) > p.arena_bytes) st = SPKV_DEVERR_RECORD;
       }
-      b = lo;
-      if (bn < (int64_t)p.seq_start[b] || bn >= (int64_t)p.seq_start[b + 1]) {
-        if (lane == 0) set_err(p.err, SPKV_DEVERR_CTX);
-        continue;
-      }
-    } else {
-      b = (int)(bn / p.n_new);
-      pos = p.start_pos[b] + (int)(bn % p.n_new);
     }
-    if (pos < 0 || pos >= p.max_pages * kPage) {
-      if (lane == 0) set_err(p.err, SPKV_DEVERR_CTX);
+    if (st) {
+      set_err(p.err, st);
       continue;
     }
-    const int pid = p.block_table[(int64_t)b * p.max_pages + pos / kPage];
-    if (pid < 0 || pid >= p.num_pages) {
-      if (lane == 0) set_err(p.err, SPKV_DEVERR_PAGE_ID);
-      continue;
+    encode_key_lane_bits(bits, p.keys + item * kD, p.arena + rec, pl.slot, p.rad_lo[pl.h], p.rad_step[pl.h],
+                         sm.pol_c2, sm.az_c2, p.err);
+    if (p.values) {  // the value row
+      const uint2 *src = reinterpret_cast<const uint2 *>(p.values + item * kD);
+      uint2 *dst = reinterpret_cast<uint2 *>(p.v_pages + (((int64_t)pl.pid * p.Hkv + pl.h) * kPage + pl.slot) * kD);
+#pragma unroll 8
+      for (int j = 0; j < kD / 4; ++j) dst[j] = src[j];
     }
-    const spkv_page_hdr hd = p.hdr[pid];
-    const int bits = hd.bits;
-    if (tier_of_bits(bits) < 0) {
-      if (lane == 0) set_err(p.err, SPKV_DEVERR_BITS);
-      continue;
-    }
-    const uint64_t rec = (uint64_t)hd.code_off16 * 16u + (uint64_t)h * rec_bytes(bits);
-    if (rec + rec_bytes(bits) > p.arena_bytes) {
-      if (lane == 0) set_err(p.err, SPKV_DEVERR_RECORD);
-      continue;
-    }
-    const int slot = pos % kPage;
-
-    encode_key_warp(p.keys + item * kD, bits, p.arena + rec, slot, p.rad_lo[h], p.rad_step[h], sm.pol_c2, sm.az_c2,
-                    sm.codes[wid], lane, p.err);
-    // ---- value row (optional)
-    if (p.values) {
-      const uint2 v = *reinterpret_cast<const uint2 *>(p.values + item * kD + 4 * lane);
-      uint16_t *dst = p.v_pages + (((int64_t)pid * p.Hkv + h) * kPage + slot) * kD + 4 * lane;
-      *reinterpret_cast<uint2 *>(dst) = v;
-    }
-    __syncwarp();
   }
 }
 
@@ -141,8 +171,10 @@ spkv_status launch_encode(const spkv_cache *cache, EncodeParams &p, cudaStream_t
   p.num_pages = cache->num_pages;
   const int sms = device_sm_count();
   if (sms <= 0) return SPKV_ERR_CUDA;
-  const int64_t want = (p.items + kEncWarps - 1) / kEncWarps;
-  const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+  // one wave of resident CTAs (3 per SM), each warp striding over the items
+  // one wave of resident CTAs (4 per SM), each thread striding over the items
+  const int64_t want = (p.items + kEncThreads - 1) / kEncThreads;
+  const int grid = (int)(want < (int64_t)sms * 4 ? want : (int64_t)sms * 4);
   encode_kernel<<<grid, kEncThreads, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
 }

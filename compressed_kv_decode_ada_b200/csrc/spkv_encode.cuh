@@ -1,84 +1,229 @@
-// spkv_encode.cuh -- one warp encodes one key into its page slot: shared by
-// the bulk encode kernel (spkv_encode_keys) and the decode kernel's fused
-// single-token append (spkv_decode_attention_append), so both write the same
-// bytes for the same key.
+// spkv_encode.cuh -- a key into its page slot: one thread per key for the
+// bulk encode kernel (spkv_encode_keys), one warp per key for the decode
+// kernel's fused single-token append (spkv_decode_attention_append); the two
+// forms do the same arithmetic, so they write the same bytes for a key.
 //
 // Method: "SPHERICAL KV: Angle-Domain Attention and Rate-Distortion Retention
 // for Efficient Long-Context Inference", technical summary section 2.1
 // (r = ||k||, phi = Phi(k^); quantised radius and packed angle codes).  Every
-// angle code is decided in fp64 from the exact squares of the bf16 inputs
-// (lane_codes); the radius code uses fp64 log2.
+// angle code is decided in fp64 from the exact squares of the bf16 inputs;
+// the radius code uses fp64 log2.
+//
+// Order of the suffix sums S_i = sum_{j >= i} x_j^2 (fixed, so that every
+// path that encodes a key rounds them alike): the key is cut into 32 groups of
+// four dims; group g's local sums are s3 = x3^2, s2 = fma(x2, x2, s3),
+// s1 = fma(x1, x1, s2), s0 = fma(x0, x0, s1) (x_k = dim 4g + k); T_32 = 0 and
+// T_g = s0 + T_(g+1); then S_(4g+k) = s_k + T_(g+1).
 #pragma once
 
 #include "spkv_common.cuh"
 
 namespace spkv {
 
-// Word w (32 bits) of a slot's bitstream, from the byte-per-angle codes.
+// The same codes as polar_code, by a search over half the edges: with
+// S > 0, the sign of x fixes the half of [0, pi] the angle lies in --
+//   x > 0: the code is the largest k in [0, 2^(b-1)) with x^2 <= S c2[k]
+//          (k = 0 always: c2[0] = 1, x^2 <= S);
+//   x < 0: the code is 2^(b-1) + the largest j in [0, 2^(b-1)) with j = 0 or
+//          x^2 >= S c2[2^(b-1) + j];
+//   x = 0: the angle is pi/2 exactly, code 2^(b-1)
+// (polar_reaches' tests, in which "x <= 0" and "x < 0" are fixed per angle;
+// c2[2^(b-1)] = 0 exactly, so k = 2^(b-1) is not reached for x > 0).
 template <int BITS>
-__device__ __forceinline__ uint32_t pack_word(const uint8_t *codes, int w) {
-  const int lo_bit = 32 * w;
-  const int a0 = lo_bit / BITS, a1 = min(127, (lo_bit + 31) / BITS);
-  uint32_t v = 0;
-  for (int a = a0; a <= a1; ++a) {
-    const int sh = a * BITS - lo_bit;
-    const uint32_t c = codes[a];
-    v |= sh >= 0 ? (c << sh) : (c >> (-sh));
+__device__ __forceinline__ int polar_code_half(double x, double S, const double *c2) {
+  constexpr int H = 1 << (BITS - 1);
+  const double x2 = x * x;
+  const bool pos = x > 0.0;
+  const double *tab = pos ? c2 : c2 + H;
+  int lo = 0, hi = H - 1;
+#pragma unroll
+  for (int it = 0; it < BITS - 1; ++it) {
+    const int mid = (lo + hi + 1) >> 1;
+    const double rhs = S * tab[mid];
+    const bool r = pos ? x2 <= rhs : x2 >= rhs;
+    lo = r ? mid : lo;
+    hi = r ? hi : mid - 1;
   }
-  return v;
+  int code = pos ? lo : H + lo;
+  code = x == 0.0 ? H : code;
+  return S == 0.0 ? 0 : code;
 }
 
-// The calling warp encodes key[0..127] (bf16 bits; lane l holds dims
-// 4l..4l+3) into slot `slot` of the (page, kv head) record at recp, whose
-// pages have bit width `bits` (a valid tier): the 127 angle codes, packed
-// LSB-first into the slot's chunk-major bitstream, and the radius byte after
-// the 256 b code bytes.  codes_smem: 128 bytes of this warp's shared memory.
-// pol_c2 / az_c2: the fp64 cos^2 edge tables (build_edge_tables).
-__device__ __forceinline__ void encode_key_warp(const uint16_t *key, int bits, uint8_t *recp, int slot, float Lf,
-                                                float Df, const double *pol_c2, const double *az_c2,
-                                                uint8_t *codes_smem, int lane, uint32_t *err) {
-  // ---- x (4 per lane); exact squares and suffix sums in fp64
-  const uint2 raw = *reinterpret_cast<const uint2 *>(key + 4 * lane);
-  double x[4], S[4];
-  lane_suffix_sums(raw, lane, x, S);
-  const double x127 = __shfl_sync(0xffffffffu, x[3], 31);
-
-  // ---- angle codes (fp64 decisions), one byte per angle in shared memory
-  int c4[4];
-  switch (bits) {
-    case 3: lane_codes<3>(x, S, x127, lane, pol_c2, az_c2, c4); break;
-    case 4: lane_codes<4>(x, S, x127, lane, pol_c2, az_c2, c4); break;
-    case 6: lane_codes<6>(x, S, x127, lane, pol_c2, az_c2, c4); break;
-    default: lane_codes<8>(x, S, x127, lane, pol_c2, az_c2, c4); break;
+// The slot's bitstream (codes LSB first, code i at bits [i b, i b + b)) is
+// built from the top code down in a 64-bit accumulator (acc = acc << b | c),
+// and word w = bits [32 w, 32 w + 32) is taken once the lowest code added
+// starts at or below bit 32 w; the four words of chunk c = w / 4 go out as one
+// 16-byte store at recp + (16 c + slot) 16 (chunk-major record layout).
+struct SlotWords {
+  uint64_t acc = 0u;
+  int w;       // next word to take (descending)
+  uint4 stage;  // the chunk being filled
+  uint8_t *recp;
+  int slot;
+  __device__ __forceinline__ SlotWords(uint8_t *r, int s, int nwords) : w(nwords - 1), recp(r), slot(s) {
+    stage = make_uint4(0u, 0u, 0u, 0u);
   }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) codes_smem[4 * lane + k] = (uint8_t)c4[k];
-  __syncwarp();
-
-  // ---- pack: lane w < 4b builds word w; store chunk-major
-  if (lane < 4 * bits) {
-    uint32_t word;
-    switch (bits) {
-      case 3: word = pack_word<3>(codes_smem, lane); break;
-      case 4: word = pack_word<4>(codes_smem, lane); break;
-      case 6: word = pack_word<6>(codes_smem, lane); break;
-      default: word = pack_word<8>(codes_smem, lane); break;
+  template <int BITS>
+  __device__ __forceinline__ void push(int i, uint32_t c) {
+    acc = (acc << BITS) | c;
+    if (i * BITS <= 32 * w) {  // word w complete (uniform across lanes that run the same key index)
+      const uint32_t word = (uint32_t)(acc >> (32 * w - i * BITS));
+      const int wic = w & 3;
+      stage.x = wic == 0 ? word : stage.x;
+      stage.y = wic == 1 ? word : stage.y;
+      stage.z = wic == 2 ? word : stage.z;
+      stage.w = wic == 3 ? word : stage.w;
+      if (wic == 0) *reinterpret_cast<uint4 *>(recp + ((w >> 2) * 16 + slot) * 16) = stage;
+      --w;
     }
-    const int chunk = lane >> 2, wic = lane & 3;
-    *reinterpret_cast<uint32_t *>(recp + (chunk * 16 + slot) * 16 + wic * 4) = word;
   }
-  // ---- radius code (lane 0 holds S_0 = ||k||^2)
+};
+
+// Four dims of a key (bf16 bits) as fp64.
+__device__ __forceinline__ void bf16x4_to_f64(uint2 raw, double (&x)[4]) {
+  x[0] = bf16_to_f64(raw.x & 0xffffu);
+  x[1] = bf16_to_f64(raw.x >> 16);
+  x[2] = bf16_to_f64(raw.y & 0xffffu);
+  x[3] = bf16_to_f64(raw.y >> 16);
+}
+
+// The calling thread encodes key[0..127] (bf16 bits, 8-byte aligned) into
+// slot `slot` of the (page, kv head) record at recp, whose pages have bit
+// width BITS: the 127 angle codes, packed LSB first into the slot's
+// chunk-major bitstream, and the radius byte after the 256 b code bytes.
+// pc2 / ac2: this tier's fp64 cos^2 edge tables (build_edge_tables).
+template <int BITS>
+__device__ __forceinline__ void encode_key_lane(const uint16_t *key, uint8_t *recp, int slot, float Lf, float Df,
+                                                const double *pc2, const double *ac2, uint32_t *err) {
+  SlotWords sw(recp, slot, 4 * BITS);
+  const uint2 *kr = reinterpret_cast<const uint2 *>(key);
+  // ---- group 31: dims 124..127 (angles 124, 125 polar, 126 the azimuth, 127 padding)
+  double x[4], s[4];
+  bf16x4_to_f64(kr[31], x);
+  s[3] = x[3] * x[3];
+  s[2] = fma(x[2], x[2], s[3]);
+  s[1] = fma(x[1], x[1], s[2]);
+  s[0] = fma(x[0], x[0], s[1]);
+  double T = s[0] + 0.0;  // T_31 (T_32 = 0)
+  sw.push<BITS>(127, 0u);
+  sw.push<BITS>(126, (uint32_t)azimuth_code<BITS>(x[2], x[3], s[2] + 0.0, ac2));
+  sw.push<BITS>(125, (uint32_t)polar_code_half<BITS>(x[1], s[1] + 0.0, pc2));
+  sw.push<BITS>(124, (uint32_t)polar_code_half<BITS>(x[0], s[0] + 0.0, pc2));
+  // ---- groups 30 .. 0, the next group's dims loaded one step ahead
+  uint2 nxt = kr[30];
+#pragma unroll 1
+  for (int g = 30; g >= 0; --g) {
+    bf16x4_to_f64(nxt, x);
+    if (g > 0) nxt = kr[g - 1];
+    s[3] = x[3] * x[3];
+    s[2] = fma(x[2], x[2], s[3]);
+    s[1] = fma(x[1], x[1], s[2]);
+    s[0] = fma(x[0], x[0], s[1]);
+    const double Tn = T;  // T_(g+1)
+    T = s[0] + Tn;        // T_g
+#pragma unroll
+    for (int k = 3; k >= 0; --k)
+      sw.push<BITS>(4 * g + k, (uint32_t)polar_code_half<BITS>(x[k], s[k] + Tn, pc2));
+  }
+  // ---- radius code from S_0 = T_0 = ||k||^2
+  int c = 0;
+  if (!(Df > 0.0f) || !isfinite(Df) || !isfinite(Lf)) {
+    set_err(err, SPKV_DEVERR_RADIUS);
+  } else if (T > 0.0) {
+    const double tr = (log2(sqrt(T)) - (double)Lf) / (double)Df + 0.5;
+    c = tr <= 0.0 ? 0 : tr >= 255.0 ? 255 : (int)floor(tr);
+  }
+  recp[256 * BITS + slot] = (uint8_t)c;
+}
+
+// encode_key_lane for the tier of `bits` (a valid tier: 3, 4, 6 or 8).
+__device__ __forceinline__ void encode_key_lane_bits(int bits, const uint16_t *key, uint8_t *recp, int slot,
+                                                     float Lf, float Df, const double *pol_c2,
+                                                     const double *az_c2, uint32_t *err) {
+  const int t = tier_of_bits(bits);
+  const double *pc2 = pol_c2 + lut_off(t), *ac2 = az_c2 + lut_off(t);
+  switch (bits) {
+    case 3: encode_key_lane<3>(key, recp, slot, Lf, Df, pc2, ac2, err); break;
+    case 4: encode_key_lane<4>(key, recp, slot, Lf, Df, pc2, ac2, err); break;
+    case 6: encode_key_lane<6>(key, recp, slot, Lf, Df, pc2, ac2, err); break;
+    default: encode_key_lane<8>(key, recp, slot, Lf, Df, pc2, ac2, err); break;
+  }
+}
+
+// The same bytes as encode_key_lane, computed by a whole warp (the fused
+// append's form, one key at a time): lane l holds dims 4l .. 4l+3 (group l)
+// and forms the group's local sums; the group suffix T_l = s0_l + T_(l+1)
+// runs down the lanes one addition at a time (the same additions, so the
+// same roundings); each lane decides its four codes, and the slot's words are
+// put together by funnel shifts across lanes.
+template <int BITS>
+__device__ __forceinline__ void encode_key_warp_seq(const uint16_t *key, uint8_t *recp, int slot, float Lf,
+                                                    float Df, const double *pc2, const double *ac2, int lane,
+                                                    uint32_t *err) {
+  double x[4], s[4];
+  bf16x4_to_f64(*reinterpret_cast<const uint2 *>(key + 4 * lane), x);
+  s[3] = x[3] * x[3];
+  s[2] = fma(x[2], x[2], s[3]);
+  s[1] = fma(x[1], x[1], s[2]);
+  s[0] = fma(x[0], x[0], s[1]);
+  double T = 0.0;  // lane l: T_l once the chain has passed it
+  if (lane == 31) T = s[0] + 0.0;
+#pragma unroll 1
+  for (int l = 30; l >= 0; --l) {
+    const double up = __shfl_sync(0xffffffffu, T, l + 1);
+    if (lane == l) T = s[0] + up;
+  }
+  double Tn = __shfl_down_sync(0xffffffffu, T, 1);  // T_(l+1)
+  if (lane == 31) Tn = 0.0;
+  uint32_t grp = 0u;  // this lane's four codes, LSB first
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int a = 4 * lane + k;
+    const double S = s[k] + Tn;
+    int c = polar_code_half<BITS>(x[k], S, pc2);
+    if (a >= 126) c = a == 126 ? azimuth_code<BITS>(x[2], x[3], S, ac2) : 0;
+    grp |= (uint32_t)c << (k * BITS);
+  }
+  // word w = bits [32 w, 32 w + 32): from the groups of lanes first ..
+  // first + SPAN - 1, first = 32 w / (4 b)
+  constexpr int GB = 4 * BITS, SPAN = BITS == 3 ? 4 : (BITS == 8 ? 1 : 2);
+  const int first = (32 * lane) / GB, off = 32 * lane - first * GB;
+  uint64_t acc = 0u;
+#pragma unroll
+  for (int j = 0; j < SPAN; ++j) {
+    const uint32_t gj = __shfl_sync(0xffffffffu, grp, min(first + j, 31));
+    acc |= (uint64_t)gj << (j * GB);
+  }
+  if (lane < GB) {
+    const int chunk = lane >> 2, wic = lane & 3;
+    *reinterpret_cast<uint32_t *>(recp + (chunk * 16 + slot) * 16 + wic * 4) = (uint32_t)(acc >> off);
+  }
+  // ---- radius code from S_0 = T_0 (lane 0)
   if (lane == 0) {
     int c = 0;
     if (!(Df > 0.0f) || !isfinite(Df) || !isfinite(Lf)) {
       set_err(err, SPKV_DEVERR_RADIUS);
-    } else if (S[0] > 0.0) {
-      const double t = (log2(sqrt(S[0])) - (double)Lf) / (double)Df + 0.5;
-      c = t <= 0.0 ? 0 : t >= 255.0 ? 255 : (int)floor(t);
+    } else if (T > 0.0) {
+      const double tr = (log2(sqrt(T)) - (double)Lf) / (double)Df + 0.5;
+      c = tr <= 0.0 ? 0 : tr >= 255.0 ? 255 : (int)floor(tr);
     }
-    recp[256 * bits + slot] = (uint8_t)c;
+    recp[256 * BITS + slot] = (uint8_t)c;
   }
   __syncwarp();
+}
+
+// encode_key_warp_seq for the tier of `bits` (a valid tier).
+__device__ __forceinline__ void encode_key_warp_seq_bits(int bits, const uint16_t *key, uint8_t *recp, int slot,
+                                                         float Lf, float Df, const double *pol_c2,
+                                                         const double *az_c2, int lane, uint32_t *err) {
+  const int t = tier_of_bits(bits);
+  const double *pc2 = pol_c2 + lut_off(t), *ac2 = az_c2 + lut_off(t);
+  switch (bits) {
+    case 3: encode_key_warp_seq<3>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
+    case 4: encode_key_warp_seq<4>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
+    case 6: encode_key_warp_seq<6>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
+    default: encode_key_warp_seq<8>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
+  }
 }
 
 }  // namespace spkv
