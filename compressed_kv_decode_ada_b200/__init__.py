@@ -8,7 +8,8 @@ loudly when the CUDA library has not been built.
 from ._lib import LIB_PATH, SpkvError, lib  # noqa: F401
 from .cache import SpkvCache  # noqa: F401
 from .ops import (alloc_workspace, debug_logits, decode_attention, decode_attention_append,  # noqa: F401
-                  decode_attention_partial, decode_attention_static_ws, decompress_then_dot, default_splits,
-                  dense_decode, encode_keys, encode_keys_packed, merge_partials, rdr_plan, rdr_workspace_bytes,
+                  decode_attention_nonuniform, decode_attention_partial, decode_attention_static_ws,
+                  decompress_then_dot, default_splits, dense_decode, encode_keys, encode_keys_nonuniform,
+                  encode_keys_packed, merge_partials, nonuniform_tables, rdr_plan, rdr_workspace_bytes,
                   workspace_bytes)
 from .rdr import allocate_packed, build_packed_cache  # noqa: F401

@@ -38,6 +38,9 @@ EXPORTS = (
     "spkv_rdr_plan",
     "spkv_encode_keys_packed",
     "spkv_nonuniform_tables",
+    "spkv_encode_keys_nonuniform",
+    "spkv_decode_nonuniform_workspace_bytes",
+    "spkv_decode_attention_nonuniform",
 )
 PARTIAL_FLOATS = 132  # floats per (sequence, query head) shard record
 DECODE_EXACT_Q = 1  # SPKV_DECODE_EXACT_Q
@@ -129,6 +132,13 @@ def _load():
                                           _P]
     L.spkv_nonuniform_tables.restype = ctypes.c_int
     L.spkv_nonuniform_tables.argtypes = [_I, _I, _P, _P, _P]
+    L.spkv_encode_keys_nonuniform.restype = ctypes.c_int
+    L.spkv_encode_keys_nonuniform.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _P, _P, _I, _I, _P, _I, _I, _P, _P]
+    L.spkv_decode_nonuniform_workspace_bytes.restype = ctypes.c_size_t
+    L.spkv_decode_nonuniform_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
+    L.spkv_decode_attention_nonuniform.restype = ctypes.c_int
+    L.spkv_decode_attention_nonuniform.argtypes = [ctypes.POINTER(SpkvCacheC), _P, _I, _I, _P, _I, _P, _I, _I, _P, _P,
+                                                   _P, _P, _I, _P, _P, ctypes.c_size_t, _I, _P]
     return L
 
 

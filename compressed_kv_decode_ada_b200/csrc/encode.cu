@@ -37,6 +37,10 @@ struct EncodeParams {
   const int32_t *seq_start, *dst_pos;  // scattered placement (start_pos unused)
   int B, n_new, max_pages;
   int64_t items;  // B * n_new * Hkv, or total_tokens * Hkv when scattered
+  // non-uniform quantiser (nullptr: the uniform one): every page must have
+  // b = nu_bits; nu_ec holds the 126 x (2^b - 1) polar edge cosines
+  const double *nu_ec;
+  int nu_bits;
 };
 
 struct EncodeSmem {
@@ -127,8 +131,17 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const EncodePara
       set_err(p.err, st);
       continue;
     }
-    encode_key_lane_bits(bits, p.keys + item * kD, p.arena + rec, pl.slot, p.rad_lo[pl.h], p.rad_step[pl.h],
-                         sm.pol_c2, sm.az_c2, p.err);
+    if (p.nu_ec) {
+      if (bits != p.nu_bits) {
+        set_err(p.err, SPKV_DEVERR_BITS);
+        continue;
+      }
+      encode_key_lane_nu_bits(bits, p.keys + item * kD, p.arena + rec, pl.slot, p.rad_lo[pl.h],
+                              p.rad_step[pl.h], sm.az_c2, p.nu_ec, p.err);
+    } else {
+      encode_key_lane_bits(bits, p.keys + item * kD, p.arena + rec, pl.slot, p.rad_lo[pl.h], p.rad_step[pl.h],
+                           sm.pol_c2, sm.az_c2, p.err);
+    }
     if (p.values) {  // the value row
       const uint2 *src = reinterpret_cast<const uint2 *>(p.values + item * kD);
       uint2 *dst = reinterpret_cast<uint2 *>(p.v_pages + (((int64_t)pl.pid * p.Hkv + pl.h) * kPage + pl.slot) * kD);
@@ -225,5 +238,32 @@ extern "C" spkv_status spkv_encode_keys_packed(const spkv_cache *cache, const ui
   p.n_new = 0;
   p.max_pages = max_pages;
   p.items = total_tokens * cache->num_kv_heads;
+  return launch_encode(cache, p, (cudaStream_t)stream);
+}
+
+extern "C" spkv_status spkv_encode_keys_nonuniform(const spkv_cache *cache, const uint16_t *keys,
+                                                   const uint16_t *values, const int32_t *start_pos, int32_t B,
+                                                   int32_t n_new, const int32_t *block_table, int32_t max_pages,
+                                                   int32_t bits, const double *edge_cos, void *stream) {
+  using namespace spkv;
+  spkv_status st = check_cache(cache);
+  if (st != SPKV_OK) return st;
+  if (B < 0 || n_new < 0 || max_pages < 0) return SPKV_ERR_INVALID_ARG;
+  if (tier_of_bits(bits) < 0) return SPKV_ERR_UNSUPPORTED;
+  if (!edge_cos || ((uintptr_t)edge_cos & 7)) return SPKV_ERR_INVALID_ARG;
+  if (B == 0 || n_new == 0) return SPKV_OK;
+  if (!keys || !start_pos || !block_table || max_pages == 0) return SPKV_ERR_INVALID_ARG;
+  if (((uintptr_t)keys & 7) || ((uintptr_t)values & 7)) return SPKV_ERR_INVALID_ARG;
+  EncodeParams p = {};
+  p.keys = keys;
+  p.values = values;
+  p.start_pos = start_pos;
+  p.block_table = block_table;
+  p.B = B;
+  p.n_new = n_new;
+  p.max_pages = max_pages;
+  p.items = (int64_t)B * n_new * cache->num_kv_heads;
+  p.nu_ec = edge_cos;
+  p.nu_bits = bits;
   return launch_encode(cache, p, (cudaStream_t)stream);
 }

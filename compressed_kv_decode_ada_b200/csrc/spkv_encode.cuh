@@ -49,6 +49,28 @@ __device__ __forceinline__ int polar_code_half(double x, double S, const double 
   return S == 0.0 ? 0 : code;
 }
 
+// Non-uniform quantiser (an f_b variant): polar angle a has its own edges,
+// ec[j - 1] = cos theta_j (j = 1 .. 2^b - 1, increasing angles), and its code
+// is the largest j whose edge it reaches (j = 0 always), by the same exact
+// test: phi >= theta <=> x <= sqrt(S) cos theta, decided on x^2 vs S cos^2
+// and the signs.
+template <int BITS>
+__device__ __forceinline__ int polar_code_nu(double x, double S, const double *ec) {
+  if (S == 0.0) return 0;
+  const double x2 = x * x;
+  int lo = 0, hi = (1 << BITS) - 1;
+#pragma unroll
+  for (int it = 0; it < BITS; ++it) {
+    const int mid = (lo + hi + 1) >> 1;
+    const double c = ec[mid - 1];
+    const double rhs = S * (c * c);
+    const bool r = c >= 0.0 ? (x <= 0.0 || x2 <= rhs) : (x < 0.0 && x2 >= rhs);
+    lo = r ? mid : lo;
+    hi = r ? hi : mid - 1;
+  }
+  return lo;
+}
+
 // The slot's bitstream (codes LSB first, code i at bits [i b, i b + b)) is
 // built from the top code down in a 64-bit accumulator (acc = acc << b | c),
 // and word w = bits [32 w, 32 w + 32) is taken once the lowest code added
@@ -92,9 +114,17 @@ __device__ __forceinline__ void bf16x4_to_f64(uint2 raw, double (&x)[4]) {
 // width BITS: the 127 angle codes, packed LSB first into the slot's
 // chunk-major bitstream, and the radius byte after the 256 b code bytes.
 // pc2 / ac2: this tier's fp64 cos^2 edge tables (build_edge_tables).
-template <int BITS>
+// NU: the non-uniform quantiser's polar codes, against nu_ec (row a: the
+// 2^b - 1 edge cosines of angle a); the azimuth and radius are unchanged.
+template <int BITS, bool NU = false>
 __device__ __forceinline__ void encode_key_lane(const uint16_t *key, uint8_t *recp, int slot, float Lf, float Df,
-                                                const double *pc2, const double *ac2, uint32_t *err) {
+                                                const double *pc2, const double *ac2, uint32_t *err,
+                                                const double *nu_ec = nullptr) {
+  constexpr int NE = (1 << BITS) - 1;
+  auto polar = [&](int a, double x, double S) -> uint32_t {
+    if constexpr (NU) return (uint32_t)polar_code_nu<BITS>(x, S, nu_ec + a * NE);
+    else return (uint32_t)polar_code_half<BITS>(x, S, pc2);
+  };
   SlotWords sw(recp, slot, 4 * BITS);
   const uint2 *kr = reinterpret_cast<const uint2 *>(key);
   // ---- group 31: dims 124..127 (angles 124, 125 polar, 126 the azimuth, 127 padding)
@@ -107,14 +137,19 @@ __device__ __forceinline__ void encode_key_lane(const uint16_t *key, uint8_t *re
   double T = s[0] + 0.0;  // T_31 (T_32 = 0)
   sw.push<BITS>(127, 0u);
   sw.push<BITS>(126, (uint32_t)azimuth_code<BITS>(x[2], x[3], s[2] + 0.0, ac2));
-  sw.push<BITS>(125, (uint32_t)polar_code_half<BITS>(x[1], s[1] + 0.0, pc2));
-  sw.push<BITS>(124, (uint32_t)polar_code_half<BITS>(x[0], s[0] + 0.0, pc2));
-  // ---- groups 30 .. 0, the next group's dims loaded one step ahead
-  uint2 nxt = kr[30];
+  sw.push<BITS>(125, polar(125, x[1], s[1] + 0.0));
+  sw.push<BITS>(124, polar(124, x[0], s[0] + 0.0));
+  // ---- groups 30 .. 0; each group's dims are loaded eight groups (two
+  // 32-byte sectors of the row) ahead, through a shift register
+  uint2 pf[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) pf[j] = kr[30 - j];
 #pragma unroll 1
   for (int g = 30; g >= 0; --g) {
-    bf16x4_to_f64(nxt, x);
-    if (g > 0) nxt = kr[g - 1];
+    bf16x4_to_f64(pf[0], x);
+#pragma unroll
+    for (int j = 0; j < 7; ++j) pf[j] = pf[j + 1];
+    pf[7] = g >= 8 ? kr[g - 8] : make_uint2(0u, 0u);
     s[3] = x[3] * x[3];
     s[2] = fma(x[2], x[2], s[3]);
     s[1] = fma(x[1], x[1], s[2]);
@@ -123,7 +158,7 @@ __device__ __forceinline__ void encode_key_lane(const uint16_t *key, uint8_t *re
     T = s[0] + Tn;        // T_g
 #pragma unroll
     for (int k = 3; k >= 0; --k)
-      sw.push<BITS>(4 * g + k, (uint32_t)polar_code_half<BITS>(x[k], s[k] + Tn, pc2));
+      sw.push<BITS>(4 * g + k, polar(4 * g + k, x[k], s[k] + Tn));
   }
   // ---- radius code from S_0 = T_0 = ||k||^2
   int c = 0;
@@ -147,6 +182,20 @@ __device__ __forceinline__ void encode_key_lane_bits(int bits, const uint16_t *k
     case 4: encode_key_lane<4>(key, recp, slot, Lf, Df, pc2, ac2, err); break;
     case 6: encode_key_lane<6>(key, recp, slot, Lf, Df, pc2, ac2, err); break;
     default: encode_key_lane<8>(key, recp, slot, Lf, Df, pc2, ac2, err); break;
+  }
+}
+
+// encode_key_lane with the non-uniform polar codes, for b = bits (a valid
+// tier); nu_ec: the 126 x (2^b - 1) edge cosines of the polar angles.
+__device__ __forceinline__ void encode_key_lane_nu_bits(int bits, const uint16_t *key, uint8_t *recp, int slot,
+                                                        float Lf, float Df, const double *az_c2,
+                                                        const double *nu_ec, uint32_t *err) {
+  const double *ac2 = az_c2 + lut_off(tier_of_bits(bits));
+  switch (bits) {
+    case 3: encode_key_lane<3, true>(key, recp, slot, Lf, Df, nullptr, ac2, err, nu_ec); break;
+    case 4: encode_key_lane<4, true>(key, recp, slot, Lf, Df, nullptr, ac2, err, nu_ec); break;
+    case 6: encode_key_lane<6, true>(key, recp, slot, Lf, Df, nullptr, ac2, err, nu_ec); break;
+    default: encode_key_lane<8, true>(key, recp, slot, Lf, Df, nullptr, ac2, err, nu_ec); break;
   }
 }
 

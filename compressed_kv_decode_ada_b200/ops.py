@@ -67,6 +67,71 @@ def encode_keys(cache: SpkvCache, keys: torch.Tensor, start_pos: torch.Tensor, b
                                _ptr(block_table), block_table.shape[1], _stream(stream)), "spkv_encode_keys")
 
 
+def encode_keys_nonuniform(cache: SpkvCache, keys: torch.Tensor, start_pos: torch.Tensor, block_table: torch.Tensor,
+                           bits: int, edge_cos: torch.Tensor, values: torch.Tensor | None = None,
+                           stream=None) -> None:
+    """spkv_encode_keys_nonuniform: as encode_keys, with the non-uniform angle
+    quantiser at b = bits (every page must have that width); edge_cos: the
+    [126, 2^b - 1] fp64 polar edge cosines (nonuniform_tables(128, bits)[0])
+    on the device."""
+    _need(keys, torch.bfloat16, "keys", 4)
+    B, n_new, hkv, d = keys.shape
+    if hkv != cache.num_kv_heads or d != HEAD_DIM:
+        raise ValueError("keys must be [B, n_new, H_kv, 128]")
+    if values is not None:
+        _need(values, torch.bfloat16, "values", 4)
+        if values.shape != keys.shape:
+            raise ValueError("values must match keys")
+    _need(start_pos, torch.int32, "start_pos", 1)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(edge_cos, torch.float64, "edge_cos", 2)
+    if start_pos.shape[0] != B or block_table.shape[0] != B:
+        raise ValueError("start_pos / block_table batch mismatch")
+    if tuple(edge_cos.shape) != (HEAD_DIM - 2, (1 << bits) - 1):
+        raise ValueError("edge_cos must be [126, 2^b - 1]")
+    c = cache.c_struct()
+    check(lib.spkv_encode_keys_nonuniform(ctypes.byref(c), _ptr(keys), _ptr(values), _ptr(start_pos), B, n_new,
+                                          _ptr(block_table), block_table.shape[1], int(bits), _ptr(edge_cos),
+                                          _stream(stream)), "spkv_encode_keys_nonuniform")
+
+
+def decode_attention_nonuniform(cache: SpkvCache, q: torch.Tensor, block_table: torch.Tensor,
+                                ctx_lens: torch.Tensor, max_ctx: int, bits: int, edge_cos: torch.Tensor,
+                                mid_cos: torch.Tensor, mid_sin: torch.Tensor, out=None, out_dtype=torch.float32,
+                                logits: torch.Tensor | None = None, ws=None, num_splits: int = 0,
+                                stream=None) -> torch.Tensor:
+    """spkv_decode_attention_nonuniform: ADA decode of a cache written by
+    encode_keys_nonuniform at b = bits; the three tables are
+    nonuniform_tables(128, bits) as fp64 device tensors.  logits (optional):
+    [B, Hq, max_ctx] fp32, filled for t < ctx_lens."""
+    _batch_checks(q, block_table, ctx_lens)
+    for t, name, shape in ((edge_cos, "edge_cos", (HEAD_DIM - 2, (1 << bits) - 1)),
+                           (mid_cos, "mid_cos", (HEAD_DIM - 2, 1 << bits)),
+                           (mid_sin, "mid_sin", (HEAD_DIM - 2, 1 << bits))):
+        _need(t, torch.float64, name, 2)
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be {shape}")
+    B, Hq, _ = q.shape
+    out = _out_buffer(out, B, Hq, out_dtype, q.device)
+    if logits is not None:
+        _need(logits, torch.float32, "logits", 3)
+    need = int(lib.spkv_decode_nonuniform_workspace_bytes(B, Hq, cache.num_kv_heads, int(max_ctx), int(num_splits),
+                                                          int(bits)))
+    if need == 0:
+        raise ValueError("invalid shape for spkv_decode_nonuniform_workspace_bytes")
+    if ws is None:
+        ws = torch.empty(need + 256, dtype=torch.uint8, device=q.device)
+    base = ws.data_ptr()
+    off = (-base) % 256  # the entry point wants a 256-byte aligned workspace
+    c = cache.c_struct()
+    check(lib.spkv_decode_attention_nonuniform(
+        ctypes.byref(c), _ptr(q), B, Hq, _ptr(block_table), block_table.shape[1], _ptr(ctx_lens), int(max_ctx),
+        int(bits), _ptr(edge_cos), _ptr(mid_cos), _ptr(mid_sin), _ptr(out), 1 if out.dtype == torch.bfloat16 else 0,
+        _ptr(logits), ctypes.c_void_p(base + off), ws.numel() - off, int(num_splits), _stream(stream)),
+        "spkv_decode_attention_nonuniform")
+    return out
+
+
 def _out_buffer(out, B, Hq, out_dtype, device):
     if out is None:
         out = torch.empty((B, Hq, HEAD_DIM), dtype=out_dtype, device=device)

@@ -404,6 +404,56 @@ SPKV_API spkv_status spkv_encode_keys_packed(const spkv_cache *cache, const uint
 SPKV_API spkv_status spkv_nonuniform_tables(int32_t d, int32_t b, double *edge_cos, double *mid_cos,
                                             double *mid_sin);
 
+/* Encode with the non-uniform angle quantiser (the tables above, d = 128):
+ * as spkv_encode_keys, except that polar angle i (i = 1..126) takes the code
+ * of the largest edge j of ITS OWN edges that it reaches (phi_i >= theta_ij
+ * <=> x_i <= sqrt(S_i) cos theta_ij, decided exactly on x_i^2 vs S_i cos^2
+ * and the signs, so an input on an edge goes to the upper cell up to the
+ * tables' 1e-12); the azimuth and the radius byte are as spkv_encode_keys.
+ *   bits      b in {3, 4, 6, 8}: every page written must have this width
+ *             (others set SPKV_DEVERR_BITS and are skipped), else
+ *             SPKV_ERR_UNSUPPORTED
+ *   edge_cos  [126 * (2^b - 1)] fp64, device, 8-byte aligned: the edge_cos
+ *             table of spkv_nonuniform_tables(128, b), row i-1 for angle i
+ * Decode such a cache with spkv_decode_attention_nonuniform. */
+SPKV_API spkv_status spkv_encode_keys_nonuniform(const spkv_cache *cache, const uint16_t *keys,
+                                                 const uint16_t *values, const int32_t *start_pos, int32_t B,
+                                                 int32_t n_new, const int32_t *block_table, int32_t max_pages,
+                                                 int32_t bits, const double *edge_cos, void *stream);
+
+/* Bytes of the workspace spkv_decode_attention_nonuniform needs (0: invalid
+ * arguments): the per-split partial records and the decode's (cos, sin)
+ * table.  num_splits 0: the default count, which queries the current
+ * device's SM count. */
+SPKV_API size_t spkv_decode_nonuniform_workspace_bytes(int32_t B, int32_t num_q_heads, int32_t num_kv_heads,
+                                                       int32_t max_ctx, int32_t num_splits, int32_t bits);
+
+/* ADA decode attention over a cache written by spkv_encode_keys_nonuniform
+ * at b = bits (every page the block tables reference below ctx_lens must
+ * have that width; others set SPKV_DEVERR_BITS and are dropped):
+ *   out[b, hq, :] = softmax_t(||q|| r~_t f_b(q, k_t) / sqrt(128)) . V
+ * with f_b the cosine of the decoded angles (cell medians: mid_cos / mid_sin
+ * of spkv_nonuniform_tables(128, b) for the polar angles, the uniform medians
+ * for the azimuth) and the query coded with the same quantiser at b.  Same
+ * paging, keep-mask, context and error rules as spkv_decode_attention.
+ *   edge_cos [126 * (2^b - 1)], mid_cos / mid_sin [126 * 2^b]: fp64, device
+ *   out      [B, Hq, 128] fp32 or bf16 (out_is_bf16), device, 16-byte aligned
+ *   logits   NULL, or [B, Hq, max_ctx] fp32 device: the logits (natural-log
+ *            units) of t < ctx_lens[b], -inf for evicted slots
+ *   ws       spkv_decode_nonuniform_workspace_bytes(...) bytes, device,
+ *            256-byte aligned (else SPKV_ERR_WORKSPACE)
+ *   num_splits  splits of each (sequence, kv head) row; 0: default
+ * Bits of b outside {3, 4, 6, 8} or G = Hq / H_kv outside {1, 2, 4, 8}:
+ * SPKV_ERR_UNSUPPORTED.  (A plain CUDA-core kernel: this variant is
+ * checked against its oracle; the tuned path is the uniform quantiser's.) */
+SPKV_API spkv_status spkv_decode_attention_nonuniform(const spkv_cache *cache, const uint16_t *q, int32_t B,
+                                                      int32_t num_q_heads, const int32_t *block_table,
+                                                      int32_t max_pages, const int32_t *ctx_lens, int32_t max_ctx,
+                                                      int32_t bits, const double *edge_cos, const double *mid_cos,
+                                                      const double *mid_sin, void *out, int32_t out_is_bf16,
+                                                      float *logits, void *ws, size_t ws_bytes, int32_t num_splits,
+                                                      void *stream);
+
 #ifdef __cplusplus
 }
 #endif

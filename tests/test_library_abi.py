@@ -119,6 +119,32 @@ def test_static_ws_argument_checks_match_decode(lib):
     assert need > m._lib.STATIC_WS_BYTES
 
 
+def test_nonuniform_host_argument_checks(lib):
+    """The non-uniform encode / decode reject bad arguments before any launch."""
+    m = lib
+    L = m.lib
+    c = _fake_cache(m)
+    enc = lambda bits, ec: L.spkv_encode_keys_nonuniform(ctypes.byref(c), 0x1000, None, 0x2000, 1, 1, 0x3000, 4,  # noqa: E731
+                                                          bits, ec, None)
+    assert enc(5, 0x4000) == 2           # b outside {3, 4, 6, 8}
+    assert enc(4, None) == 1             # no edge table
+    assert enc(4, 0x4004) == 1           # misaligned edge table
+
+    def dec(Hq=4, bits=4, ec=0x4000, ws=0x100000, ws_bytes=1 << 24, splits=2, B=1):
+        return L.spkv_decode_attention_nonuniform(ctypes.byref(c), 0x60000, B, Hq, 0x70000, 8, 0x80000, 128, bits,
+                                                  ec, 0x5000, 0x6000, 0x90000, 0, None, ws, ws_bytes, splits, None)
+    assert dec(Hq=6) == 2                # G = 3
+    assert dec(bits=7) == 2
+    assert dec(ec=None) == 1
+    assert dec(ws=0x100010) == 3         # workspace not 256-byte aligned
+    assert dec(ws_bytes=16) == 3         # workspace too small
+    assert dec(B=0) == 0                 # empty batch
+    # explicit split count: no device query
+    want = ((2 * 1 * 4 * 132 * 4 + 255) // 256) * 256 + 127 * 16 * 8
+    assert L.spkv_decode_nonuniform_workspace_bytes(1, 4, 2, 128, 2, 4) == want
+    assert L.spkv_decode_nonuniform_workspace_bytes(1, 4, 2, 128, 2, 5) == 0
+
+
 def test_workspace_formula(lib):
     # (C + B H_kv) segments x 6 consumer-warp slots x G partials of 132 floats
     # (rounded to 16 bytes), then one 4-byte row counter per kv row (rounded)

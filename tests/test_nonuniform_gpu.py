@@ -1,0 +1,147 @@
+"""GPU <-> oracle parity of the non-uniform angle quantiser (an f_b variant:
+equal-probability cells of each polar angle's sin^(d-1-i) law, medians for
+reconstruction, uniform azimuth; oracle/nonuniform.py).
+
+Codes: the GPU decides phi_i >= theta_ij exactly against the host tables'
+edges (accurate to 1e-12), the oracle decides floor(2^b F_i(phi_i)) on the
+probability scale; codes must be equal except on a cell edge (the oracle's
+scaled position within 1e-9 of an integer), and those must stay below 1e-6 of
+all codes.  Logits: |d f_b| <= 1e-4 (tokens whose codes agree).  Outputs:
+<= 2e-3 absolute.  The oracle encodes the keys itself."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import nonuniform as onu
+from tests import helpers
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 2e-3
+FB_TOL = 1e-4
+EDGE_REL = 1e-9
+LLAMA = "llama3_8b_b8_h32x8_t32768_b4"
+
+
+@pytest.fixture(scope="module")
+def spkv():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import compressed_kv_decode_ada_b200 as m
+    from compressed_kv_decode_ada_b200 import synthetic
+
+    return m, synthetic
+
+
+def _tables(m, bits):
+    ec, mc, ms = m.ops.nonuniform_tables(128, bits)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    return dev(ec), dev(mc), dev(ms)
+
+
+def _build(spkv, bits, **kw):
+    """A workload whose every page has b = bits, encoded with the non-uniform quantiser."""
+    m, synthetic = spkv
+    wl = synthetic.make_workload(LLAMA, device="cuda", **kw)
+    wl.page_bits = np.full(wl.num_pages, bits, np.int64)
+    cache = m.SpkvCache(wl.num_pages, wl.Hkv, wl.page_bits, wl.rad_lo, wl.rad_step, keep_mask=wl.keep_mask)
+    ec, mc, ms = _tables(m, bits)
+    for b in range(wl.B):
+        s, n = int(wl.seq_off[b]), int(wl.ctx[b])
+        if n:
+            m.encode_keys_nonuniform(cache, wl.keys[s:s + n].unsqueeze(0).contiguous(),
+                                     torch.zeros(1, dtype=torch.int32, device="cuda"),
+                                     wl.block_table[b:b + 1].contiguous(), bits, ec,
+                                     values=wl.values[s:s + n].unsqueeze(0).contiguous())
+    torch.cuda.synchronize()
+    assert cache.error_flags() == 0
+    wl.extras["code_offset"] = cache.page_code_offset
+    return wl, cache, (ec, mc, ms)
+
+
+def _positions(keys_bits, bits, L, D):
+    """The oracle's scaled positions: 2^b F_i(phi_i) of the polar angles,
+    phi 2^b / 2 pi of the azimuth, and the radius code's (floor = code)."""
+    x = oracle.bf16_to_f64(keys_bits)
+    T = x.shape[0]
+    n = 1 << bits
+    apos = np.empty((T, 127))
+    for t in range(T):
+        phi = oracle.angles(x[t])
+        for j in range(126):
+            apos[t, j] = n * float(onu.polar_cdf(phi[j], 128, j + 1))
+        apos[t, 126] = phi[126] * n / (2.0 * math.pi)
+    r = np.linalg.norm(x, axis=1)
+    with np.errstate(divide="ignore"):
+        rpos = (np.log2(r) - L) / D + 0.5
+    return apos, rpos
+
+
+def _oracle_group(wl, b, h, bits):
+    L, D = float(wl.rad_lo[h]), float(wl.rad_step[h])
+    codes, rc = onu.encode(wl.keys_bits(b, h), bits, L, D)
+    return codes, rc, L, D
+
+
+@pytest.mark.parametrize("bits", [3, 4, 6, 8])
+def test_nonuniform_encode_codes_match_the_oracle(spkv, bits):
+    wl, cache, _ = _build(spkv, bits, B=2, ctx=[150, 37], Hq=8, Hkv=2)
+    arena = cache.arena.cpu().numpy()
+    n_codes = n_edge_mismatch = 0
+    for b, h in helpers.all_groups(wl):
+        gc, gr, pads = helpers.gpu_codes_for_seq(arena, wl, b, h)
+        oc, orc, L, D = _oracle_group(wl, b, h, bits)
+        apos, rpos = _positions(wl.keys_bits(b, h), bits, L, D)
+        ea, er = helpers.near_integer(apos, EDGE_REL), helpers.near_integer(rpos, EDGE_REL)
+        assert not ((gc != oc) & ~ea).any(), np.argwhere((gc != oc) & ~ea)[:5]
+        assert not ((gr != orc) & ~er).any()
+        assert np.all(pads == 0)
+        n_codes += oc.size + orc.size
+        n_edge_mismatch += int(((gc != oc) & ea).sum() + ((gr != orc) & er).sum())
+    assert n_edge_mismatch <= max(1, 1e-6 * n_codes), (n_edge_mismatch, n_codes)
+
+
+@pytest.mark.parametrize("bits,kw", [
+    (4, dict(B=2, ctx=[300, 77], Hq=8, Hkv=2)),       # G = 4, ragged tails
+    (3, dict(B=2, ctx=[129, 16], Hq=4, Hkv=2)),       # G = 2, a one-page context
+    (6, dict(B=1, ctx=[200], Hq=16, Hkv=2)),          # G = 8
+    (8, dict(B=2, ctx=[90, 33], Hq=2, Hkv=2)),        # G = 1
+])
+def test_nonuniform_decode_matches_the_oracle(spkv, bits, kw):
+    m = spkv[0]
+    wl, cache, (ec, mc, ms) = _build(spkv, bits, **kw)
+    lg = torch.full((wl.B, wl.Hq, wl.max_ctx), float("nan"), device="cuda")
+    out = m.decode_attention_nonuniform(cache, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx, bits, ec, mc, ms,
+                                        logits=lg)
+    torch.cuda.synchronize()
+    assert cache.error_flags() == 0
+    out, lg = out.cpu().numpy(), lg.cpu().numpy()
+    arena = cache.arena.cpu().numpy()
+    err = 0.0
+    for b, h in helpers.all_groups(wl):
+        n = int(wl.ctx[b])
+        oc, rc, L, D = _oracle_group(wl, b, h, bits)
+        keep = wl.keep_of(b)
+        want = onu.ada_group(wl.q_bits(b, h), oc, bits, rc, L, D, wl.values_bits(b, h), keep=keep)
+        err = max(err, float(np.abs(out[b, h * wl.G:(h + 1) * wl.G] - want).max()))
+        # logits: ||q|| r~ f_b / sqrt(d) with the oracle's decoded vectors
+        gc, _, _ = helpers.gpu_codes_for_seq(arena, wl, b, h)
+        same = np.all(gc == oc, axis=1)
+        uk = np.stack([onu.unit_from_codes(oc[t], bits) for t in range(n)])
+        r = np.array([oracle.radius_value(int(c), L, D) for c in rc])
+        q = oracle.bf16_to_f64(wl.q_bits(b, h))
+        for g in range(wl.G):
+            qn = float(np.linalg.norm(q[g]))
+            uq = onu.unit_from_codes(onu.codes_from_angles(oracle.angles(q[g]), bits), bits)
+            ref = qn * r * (uk @ uq) / math.sqrt(128.0)
+            got = lg[b, h * wl.G + g, :n].astype(np.float64)
+            live = np.asarray(keep, bool)[:n] if keep is not None else np.ones(n, bool)
+            assert np.all(np.isinf(got[~live]))
+            sel = live & same
+            scale = qn * r[sel] / math.sqrt(128.0)
+            d = np.abs(got[sel] - ref[sel]) / np.maximum(scale, 1e-30)
+            assert d.max() <= FB_TOL, d.max()
+    assert err <= OUT_TOL, err
