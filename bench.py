@@ -254,6 +254,8 @@ def run_spkv(args, rank, world, local):
     extras = {}
     if rank == 0 and args.compare:
         extras = compare_paths(args, spkv, workload, wl, cache, ctx, max_ctx, splits, ws, stream, dev)
+        if args.compare_workloads:
+            extras["workloads"] = compare_workloads(args, spkv, workload, synthetic, stream, dev, _peaks()[0])
 
     tokens = wl.kv_tokens
     bytes_step = synthetic.ada_step_bytes(wl)
@@ -374,6 +376,54 @@ def compare_paths(args, spkv, workload, wl, cache, ctx, max_ctx, splits, ws, str
     res["rdr_plan_tokens_per_s"] = ntok / (rdr_ms * 1e-3)
     res["rdr_plan_key_bytes_gbs"] = wl.keys.numel() * 2 / (rdr_ms * 1e-3) / 1e9
     return res
+
+
+def compare_workloads(args, spkv, workload, synthetic, stream, dev, peak):
+    """The other full-size workloads of the method's evaluation (128K single
+    sequence, the 70B shape with G = 8, the ragged mixed-tier batch with
+    evictions), each in the bench's launch configuration: ADA decode and
+    dense decode time, ADA achieved GB/s and its fraction of the peak, and the
+    bulk encode of the workload's keys (with values)."""
+    import torch
+
+    n = max(5, args.compare_steps)
+
+    def timeit(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n
+
+    out = {}
+    for name in (synthetic.LONG_128K, synthetic.SHAPE_70B, synthetic.RAGGED_RDR):
+        if name == args.workload:
+            continue
+        wl = synthetic.make_workload(name, device=dev)
+        cache = workload.build_cache(wl)
+        ctx = wl.ctx_tensor()
+        ws = spkv.alloc_workspace(wl.B, wl.Hq, wl.Hkv, wl.max_ctx, 0, device=dev)
+        ada_ms = timeit(lambda: spkv.decode_attention(cache, wl.q, wl.block_table, ctx, wl.max_ctx, ws=ws,
+                                                      stream=stream))
+        gbs = synthetic.ada_step_bytes(wl) / (ada_ms * 1e-3) / 1e9
+        kp, vp = workload.dense_pages(wl)
+        dense_ms = timeit(lambda: spkv.dense_decode(kp, vp, wl.q, wl.block_table, ctx, wl.max_ctx, ws=ws,
+                                                    stream=stream))
+        del kp, vp
+        enc_ms = timeit(lambda: workload.prefill(cache, wl))
+        if cache.error_flags():
+            raise RuntimeError(f"{name}: device error flags {cache.error_flags():#x}")
+        out[name] = {"ada_decode_ms": ada_ms, "ada_achieved_gbs": gbs, "ada_frac_of_peak": gbs / peak,
+                     "ada_kv_tokens_per_s": wl.kv_tokens / (ada_ms * 1e-3), "dense_decode_ms": dense_ms,
+                     "ada_speedup_vs_dense": dense_ms / ada_ms, "encode_ms": enc_ms,
+                     "encode_keys_per_s": wl.kv_tokens * wl.Hkv / (enc_ms * 1e-3)}
+        del cache, ws, wl
+        torch.cuda.empty_cache()
+    return out
 
 
 def decode_code_hash() -> str:
@@ -551,6 +601,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--compare", type=int, default=1)
     ap.add_argument("--compare-steps", type=int, default=50)
+    ap.add_argument("--compare-workloads", type=int, default=1,
+                    help="also time the other full-size workloads (128K, 70B shape, ragged mixed tiers)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-only", choices=["ada", "dense", "dtd", "encode"], default=None,

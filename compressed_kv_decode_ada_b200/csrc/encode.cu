@@ -23,6 +23,7 @@ namespace spkv {
 namespace {
 
 constexpr int kEncThreads = 256;
+constexpr int64_t kEncWarpItems = 512;  // up to this many items: a warp per key
 
 struct EncodeParams {
   uint8_t *arena;
@@ -41,11 +42,6 @@ struct EncodeParams {
   // b = nu_bits; nu_ec holds the 126 x (2^b - 1) polar edge cosines
   const double *nu_ec;
   int nu_bits;
-};
-
-struct EncodeSmem {
-  double pol_c2[kLutEntries];
-  double az_c2[kLutEntries];
 };
 
 // Where item (key, kv head) `item` goes: its kv head, page and slot, or the
@@ -104,50 +100,110 @@ __device__ __forceinline__ EncPlace enc_place(const EncodeParams &p, int64_t ite
   return pl;
 }
 
-// One thread per item: its placement, its page header, the key's codes
-// (encode_key_lane) and its value row.
-__global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const EncodeParams p) {
-  __shared__ EncodeSmem sm;
+// Checks of an item's page header: its bit width and record offset, or the
+// device-error bits that rule it out.
+__device__ __forceinline__ uint32_t enc_record(const EncodeParams &p, const EncPlace &pl, int &bits, uint64_t &rec) {
+  if (pl.st) return pl.st;
+  const spkv_page_hdr hd = p.hdr[pl.pid];
+  bits = hd.bits;
+  if (tier_of_bits(bits) < 0) return SPKV_DEVERR_BITS;
+  if (p.nu_ec && bits != p.nu_bits) return SPKV_DEVERR_BITS;
+  rec = (uint64_t)hd.code_off16 * 16u + (uint64_t)pl.h * rec_bytes(bits);
+  if (rec + rec_bytes(bits) > p.arena_bytes) return SPKV_DEVERR_RECORD;
+  return 0u;
+}
+
+// Bulk encode: each warp takes 32 consecutive items at a time, one per lane.
+// The 32 key rows (8 KB, contiguous) come into the warp's shared-memory
+// stage with coalesced loads (rows 264 bytes apart, so the lanes' 8-byte
+// reads of their own rows fall in different bank pairs); each lane encodes
+// its key from there (encode_key_lane); the value rows are copied one row at
+// a time by the whole warp (coalesced 256-byte reads and writes).
+constexpr int kEncRowStride = 264;  // bytes per staged key row
+struct EncodeSmem {
+  double pol_c2[kLutEntries];
+  double az_c2[kLutEntries];
+  alignas(16) uint8_t rows[kEncThreads / 32][32 * kEncRowStride];
+};
+
+__global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const EncodeParams p) {
+  extern __shared__ __align__(16) uint8_t enc_smem_raw[];
+  EncodeSmem &sm = *reinterpret_cast<EncodeSmem *>(enc_smem_raw);
   build_edge_tables(sm.pol_c2, sm.az_c2, threadIdx.x, kEncThreads);
   __syncthreads();
-  const int64_t step = (int64_t)gridDim.x * kEncThreads;
-  for (int64_t item = (int64_t)blockIdx.x * kEncThreads + threadIdx.x; item < p.items; item += step) {
-    const EncPlace pl = enc_place(p, item);
-    if (pl.skip) continue;
-    uint32_t st = pl.st;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  uint8_t *stage = sm.rows[wid];
+  const int64_t nbatch = (p.items + 31) / 32;
+  const int64_t wstep = (int64_t)gridDim.x * (kEncThreads / 32);
+  for (int64_t bt = (int64_t)blockIdx.x * (kEncThreads / 32) + wid; bt < nbatch; bt += wstep) {
+    const int64_t first = bt * 32;
+    const int cnt = p.items - first < 32 ? (int)(p.items - first) : 32;
+    // ---- the batch's key rows into the stage (8-byte pieces; rows past the
+    // end of the batch are not read)
+    const uint2 *ksrc = reinterpret_cast<const uint2 *>(p.keys + first * kD);
+    for (int e = lane; e < cnt * (kD / 4); e += 32) {
+      const int r = e >> 5, c = e & 31;
+      *reinterpret_cast<uint2 *>(stage + r * kEncRowStride + c * 8) = ksrc[e];
+    }
+    __syncwarp();
+    // ---- this lane's item
+    const int64_t item = first + lane;
+    EncPlace pl{0, -1, 0, 0u, true};
     int bits = 0;
     uint64_t rec = 0;
-    if (!st) {
-      const spkv_page_hdr hd = p.hdr[pl.pid];
-      bits = hd.bits;
-      if (tier_of_bits(bits) < 0) {
-        st = SPKV_DEVERR_BITS;
-      } else {
-        rec = (uint64_t)hd.code_off16 * 16u + (uint64_t)pl.h * rec_bytes(bits);
-        if (rec + rec_bytes(bits) > p.arena_bytes) st = SPKV_DEVERR_RECORD;
+    uint32_t st = 0u;
+    if (lane < cnt) {
+      pl = enc_place(p, item);
+      if (!pl.skip) st = enc_record(p, pl, bits, rec);
+    }
+    const bool go = lane < cnt && !pl.skip && !st;
+    if (st) set_err(p.err, st);
+    const uint16_t *krow = reinterpret_cast<const uint16_t *>(stage + lane * kEncRowStride);
+    if (go) {
+      if (p.nu_ec)
+        encode_key_lane_nu_bits(bits, krow, p.arena + rec, pl.slot, p.rad_lo[pl.h], p.rad_step[pl.h], sm.az_c2,
+                                p.nu_ec, p.err);
+      else
+        encode_key_lane_bits(bits, krow, p.arena + rec, pl.slot, p.rad_lo[pl.h], p.rad_step[pl.h], sm.pol_c2,
+                             sm.az_c2, p.err);
+    }
+    // ---- the value rows, one row per step, the whole warp on each
+    if (p.values) {
+      int64_t dst_row = go ? (((int64_t)pl.pid * p.Hkv + pl.h) * kPage + pl.slot) * kD : -1;
+      for (int j = 0; j < cnt; ++j) {
+        const int64_t dr = __shfl_sync(0xffffffffu, dst_row, j);
+        if (dr < 0) continue;  // warp-uniform
+        const uint2 v = *reinterpret_cast<const uint2 *>(p.values + (first + j) * kD + 4 * lane);
+        *reinterpret_cast<uint2 *>(p.v_pages + dr + 4 * lane) = v;
       }
     }
-    if (st) {
-      set_err(p.err, st);
-      continue;
-    }
-    if (p.nu_ec) {
-      if (bits != p.nu_bits) {
-        set_err(p.err, SPKV_DEVERR_BITS);
-        continue;
-      }
-      encode_key_lane_nu_bits(bits, p.keys + item * kD, p.arena + rec, pl.slot, p.rad_lo[pl.h],
-                              p.rad_step[pl.h], sm.az_c2, p.nu_ec, p.err);
-    } else {
-      encode_key_lane_bits(bits, p.keys + item * kD, p.arena + rec, pl.slot, p.rad_lo[pl.h], p.rad_step[pl.h],
-                           sm.pol_c2, sm.az_c2, p.err);
-    }
-    if (p.values) {  // the value row
-      const uint2 *src = reinterpret_cast<const uint2 *>(p.values + item * kD);
-      uint2 *dst = reinterpret_cast<uint2 *>(p.v_pages + (((int64_t)pl.pid * p.Hkv + pl.h) * kPage + pl.slot) * kD);
-#pragma unroll 8
-      for (int j = 0; j < kD / 4; ++j) dst[j] = src[j];
-    }
+    __syncwarp();
+  }
+}
+
+// Few items (a decode step's appends): one warp per key, the warp form of
+// the same arithmetic (encode_key_warp_seq), so no thread runs a whole key.
+__global__ void __launch_bounds__(kEncThreads) encode_kernel_warp(const EncodeParams p) {
+  __shared__ double pol_c2[kLutEntries], az_c2[kLutEntries];
+  build_edge_tables(pol_c2, az_c2, threadIdx.x, kEncThreads);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * (kEncThreads / 32) + (threadIdx.x >> 5);
+  if (item >= p.items) return;
+  const EncPlace pl = enc_place(p, item);
+  if (pl.skip) return;
+  int bits = 0;
+  uint64_t rec = 0;
+  const uint32_t st = enc_record(p, pl, bits, rec);
+  if (st) {
+    if (lane == 0) set_err(p.err, st);
+    return;
+  }
+  encode_key_warp_seq_bits(bits, p.keys + item * kD, p.arena + rec, pl.slot, p.rad_lo[pl.h], p.rad_step[pl.h],
+                           pol_c2, az_c2, lane, p.err);
+  if (p.values) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(p.values + item * kD + 4 * lane);
+    *reinterpret_cast<uint2 *>(p.v_pages + (((int64_t)pl.pid * p.Hkv + pl.h) * kPage + pl.slot) * kD + 4 * lane) = v;
   }
 }
 
@@ -184,11 +240,25 @@ spkv_status launch_encode(const spkv_cache *cache, EncodeParams &p, cudaStream_t
   p.num_pages = cache->num_pages;
   const int sms = device_sm_count();
   if (sms <= 0) return SPKV_ERR_CUDA;
-  // one wave of resident CTAs (3 per SM), each warp striding over the items
-  // one wave of resident CTAs (4 per SM), each thread striding over the items
-  const int64_t want = (p.items + kEncThreads - 1) / kEncThreads;
-  const int grid = (int)(want < (int64_t)sms * 4 ? want : (int64_t)sms * 4);
-  encode_kernel<<<grid, kEncThreads, 0, stream>>>(p);
+  if (!p.nu_ec && p.items <= kEncWarpItems) {  // a decode step's appends: a warp per key
+    const int grid = (int)((p.items + kEncThreads / 32 - 1) / (kEncThreads / 32));
+    encode_kernel_warp<<<grid, kEncThreads, 0, stream>>>(p);
+  } else {
+    static bool configured[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SPKV_ERR_CUDA;
+    if (!configured[dev]) {
+      if (cudaFuncSetAttribute(encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)sizeof(EncodeSmem)) != cudaSuccess)
+        return SPKV_ERR_CUDA;
+      configured[dev] = true;
+    }
+    // one wave of resident CTAs (3 per SM), each warp striding over batches of 32 items
+    const int64_t batches = (p.items + 31) / 32;
+    const int64_t want = (batches + kEncThreads / 32 - 1) / (kEncThreads / 32);
+    const int grid = (int)(want < (int64_t)sms * 3 ? want : (int64_t)sms * 3);
+    encode_kernel<<<grid, kEncThreads, sizeof(EncodeSmem), stream>>>(p);
+  }
   return cudaGetLastError() == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
 }
 

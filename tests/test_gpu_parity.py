@@ -93,6 +93,29 @@ def test_encode_append_in_steps_matches_one_shot(spkv):
     assert torch.equal(cache2.v_pages, cache.v_pages)
 
 
+def test_encode_thread_and_warp_forms_write_the_same_bytes(spkv):
+    """Bulk encode runs one thread per key for large calls and one warp per key
+    for a few keys (decode-step appends); the two forms must write the same
+    bytes: one call of 2,800 keys vs the same keys 8 tokens (64 keys) at a time."""
+    m, synthetic, workload = spkv
+    wl = synthetic.make_workload(RAGGED, device="cuda", B=1, ctx=[350], mask=False)
+    one = m.SpkvCache(wl.num_pages, wl.Hkv, wl.page_bits, wl.rad_lo, wl.rad_step)
+    steps = m.SpkvCache(wl.num_pages, wl.Hkv, wl.page_bits, wl.rad_lo, wl.rad_step)
+    n = int(wl.ctx[0])
+    bt = wl.block_table[0:1].contiguous()
+    m.encode_keys(one, wl.keys[:n].unsqueeze(0), torch.zeros(1, dtype=torch.int32, device="cuda"), bt,
+                  values=wl.values[:n].unsqueeze(0))
+    for pos in range(0, n, 8):
+        k = min(8, n - pos)
+        m.encode_keys(steps, wl.keys[pos:pos + k].unsqueeze(0), torch.tensor([pos], dtype=torch.int32, device="cuda"),
+                      bt, values=wl.values[pos:pos + k].unsqueeze(0))
+    torch.cuda.synchronize()
+    assert one.error_flags() == 0 and steps.error_flags() == 0
+    assert len(set(int(b) for b in wl.page_bits)) > 1  # several tiers
+    assert torch.equal(one.arena, steps.arena)
+    assert torch.equal(one.v_pages, steps.v_pages)
+
+
 def _last_tokens(wl):
     idx = torch.tensor([int(wl.seq_off[b]) + int(wl.ctx[b]) - 1 for b in range(wl.B)], device=wl.keys.device)
     return wl.keys[idx].contiguous(), wl.values[idx].contiguous()
