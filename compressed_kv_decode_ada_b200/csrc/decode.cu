@@ -1339,38 +1339,47 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
 // partial_out (optional): instead of out, the row's own partial record
 // (M, L, 0, 0, o[128]) with o = out, L = sum_s 2^(m_s - M) l_s, for a later
 // merge across shards of the sequences' pages (spkv_merge_partials).
+constexpr int kMergeThreads = 256;  // 8 warps per (sequence, query head)
 template <int G>
-__global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint32_t *row_done, int C, int NCW,
-                                                    const int32_t *ctx_lens, int B, int Hkv, int Hq, int max_ctx,
-                                                    int max_pages, void *out, int out_bf16, uint32_t *err,
-                                                    float *partial_out) {
-  constexpr int kChunk = 256;  // partials per pass
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float *ws, const uint32_t *row_done, int C,
+                                                              int NCW, const int32_t *ctx_lens, int B, int Hkv,
+                                                              int Hq, int max_ctx, int max_pages, void *out,
+                                                              int out_bf16, uint32_t *err, float *partial_out) {
+  constexpr int kWarps = kMergeThreads / 32, kChunk = kMergeThreads, kBatch = 8;
   __shared__ float wgt[kChunk];
   __shared__ float lsh[kChunk];
   __shared__ int64_t off[kChunk];
-  __shared__ float mred[4];
-  __shared__ uint32_t nred[4];
+  __shared__ float mred[kWarps];
+  __shared__ uint32_t nred[kWarps];
+  __shared__ __align__(16) float accw[kWarps][kD];
+  __shared__ float denw[kWarps];
   const int hq = blockIdx.x % Hq, b = blockIdx.x / Hq;
   const int h = hq / G, g = hq % G, bh = b * Hkv + h;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   __shared__ int32_t Psh[kMaxB + 1];
-  __shared__ int32_t pscr[8];
-  build_prefix(ctx_lens, B, Hkv, max_ctx, max_pages, nullptr, Psh, pscr, tid, 128);
+  __shared__ int32_t pscr[kWarps + 1];
+  build_prefix(ctx_lens, B, Hkv, max_ctx, max_pages, nullptr, Psh, pscr, tid, kMergeThreads);
   const Partition part(Psh, B, Hkv, C);
   const int np = (Psh[b + 1] - Psh[b]) / Hkv;
-  float num = 0.f, den = 0.f, Mrow = kNegInf;
+  // lane l of every warp accumulates dims 4 l .. 4 l + 3 over the warp's share
+  // of the partials; the warps' sums are added at the end
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f, Mrow = kNegInf;
   if (np > 0) {
     const int64_t a = (int64_t)Psh[b] + (int64_t)h * np, e = a + np;
     const int64_t cf = part.split_of(a, bh), cl = part.split_of(e - 1, bh);
     // splits that hold units of the row (every split in [cf, cl] but empty ones)
     uint32_t live = 0;
-    for (int64_t cc = cf + tid; cc <= cl; cc += 128)
+    for (int64_t cc = cf + tid; cc <= cl; cc += kMergeThreads)
       live += part.live_in_row(cc, cf, cl) ? 1u : 0u;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) live += __shfl_xor_sync(0xffffffffu, live, o);
     if (lane == 0) nred[wid] = live;
     __syncthreads();
-    const uint32_t expected = (nred[0] + nred[1] + nred[2] + nred[3]) * (uint32_t)NCW;
+    uint32_t nlive = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) nlive += nred[w];
+    const uint32_t expected = nlive * (uint32_t)NCW;
     if (tid == 0) {
       const uint64_t t0 = globaltimer_ns();
       uint32_t seen;
@@ -1388,7 +1397,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint3
     const int64_t nparts = (cl - cf + 1) * NCW;
     float M = kNegInf;
     // pass 1: the max over all partials
-    for (int64_t base = 0; base < nparts; base += 128) {
+    for (int64_t base = 0; base < nparts; base += kMergeThreads) {
       float mm = kNegInf;
       if (base + tid < nparts) {
         const int64_t cc = cf + (base + tid) / NCW;
@@ -1402,11 +1411,14 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint3
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     if (lane == 0) mred[wid] = M;
     __syncthreads();
-    M = fmaxf(fmaxf(mred[0], mred[1]), fmaxf(mred[2], mred[3]));
+    M = mred[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) M = fmaxf(M, mred[w]);
     Mrow = M;
     if (M != kNegInf) {
       for (int64_t base = 0; base < nparts; base += kChunk) {
-        for (int i = tid; i < kChunk; i += 128) {
+        {  // the chunk's weights 2^(m - M), sums l and record offsets (-1: no weight)
+          const int i = tid;
           float wv = 0.f, lv = 0.f;
           int64_t o = -1;
           if (base + i < nparts) {
@@ -1429,22 +1441,49 @@ __global__ void __launch_bounds__(128) merge_kernel(const float *ws, const uint3
         }
         __syncthreads();
         const int n = (int)min((int64_t)kChunk, nparts - base);
-#pragma unroll 8
-        for (int i = 0; i < n; ++i) {
-          if (off[i] >= 0) {
-            num = fmaf(wgt[i], __ldcg(ws + off[i] + 4 + tid), num);
-            den = fmaf(wgt[i], lsh[i], den);
+        // warp w takes partials w, w + 8, ...; kBatch loads in flight per lane
+        for (int i0 = wid; i0 < n; i0 += kWarps * kBatch) {
+          float4 v[kBatch];
+          float wv[kBatch];
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            const int i = i0 + k * kWarps;
+            const int64_t o = i < n ? off[i] : -1;
+            wv[k] = 0.f;
+            v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (o >= 0) {
+              wv[k] = wgt[i];
+              den = fmaf(wv[k], lsh[i], den);
+              v[k] = __ldcg(reinterpret_cast<const float4 *>(ws + o + 4) + lane);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            acc.x = fmaf(wv[k], v[k].x, acc.x);
+            acc.y = fmaf(wv[k], v[k].y, acc.y);
+            acc.z = fmaf(wv[k], v[k].z, acc.z);
+            acc.w = fmaf(wv[k], v[k].w, acc.w);
           }
         }
         __syncthreads();
       }
     }
   }
-  const float res = den > 0.f ? num / den : 0.f;
+  reinterpret_cast<float4 *>(accw[wid])[lane] = acc;
+  if (lane == 0) denw[wid] = den;
+  __syncthreads();
+  if (tid >= kD) return;
+  float num = 0.f, dsum = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    num += accw[w][tid];
+    dsum += denw[w];
+  }
+  const float res = dsum > 0.f ? num / dsum : 0.f;
   if (partial_out) {
     float *pr = partial_out + ((int64_t)b * Hq + hq) * kPartial;
     pr[4 + tid] = res;
-    if (tid == 0) *reinterpret_cast<float4 *>(pr) = make_float4(den > 0.f ? Mrow : kNegInf, den, 0.f, 0.f);
+    if (tid == 0) *reinterpret_cast<float4 *>(pr) = make_float4(dsum > 0.f ? Mrow : kNegInf, dsum, 0.f, 0.f);
     return;
   }
   const int64_t o = ((int64_t)b * Hq + hq) * kD + tid;
@@ -1673,7 +1712,7 @@ spkv_status launch_g(const DecodeArgs &a, const CUtensorMap &vmap, cudaStream_t 
   if (cudaGetLastError() != cudaSuccess) return SPKV_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.sp.B * a.sp.Hq));
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(kMergeThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
