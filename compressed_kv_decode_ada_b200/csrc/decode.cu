@@ -543,13 +543,17 @@ __device__ __forceinline__ void ada_2page_f4(const uint8_t *recA, const uint8_t 
 }
 
 // Pair path for any width b (used for b = 3, 6, 8; b = 4 has ada_2page_f4):
-// a rolled loop of two iterations, each decoding 32 fields of both pages --
-// 32 b bits = b whole words of the slot's stream, loaded per iteration -- so
-// the loop body stays one granule long whatever b is.
+// a rolled loop over the 64 fields of the lane's half, NIT iterations of
+// 64 / NIT fields of both pages -- 64 b / NIT bits = whole words of the
+// slot's stream, loaded per iteration -- so the loop body stays short
+// (b = 3: two iterations of 32 fields; b = 6, 8: four of 16).
 template <int BITS, int G, int QT_HALF>
 __device__ __forceinline__ void ada_2page_gen(const uint8_t *recA, const uint8_t *recB, const float *qt,
                                               const float2 *lpol, const float2 *laz, int lane, float (&fA)[G],
                                               float (&fB)[G]) {
+  constexpr int NIT = BITS == 3 ? 2 : 4;
+  constexpr int FPI = 64 / NIT, PPI = FPI / 2, WPI = FPI * BITS / 32;  // fields, pairs, words per iteration
+  static_assert(FPI * BITS % 32 == 0, "an iteration covers whole words");
   const int t = lane & 15, half = lane >> 4;
   const float *qh = qt + half * QT_HALF;
   const uint32_t *ra32 = reinterpret_cast<const uint32_t *>(recA);
@@ -561,26 +565,26 @@ __device__ __forceinline__ void ada_2page_gen(const uint8_t *recA, const uint8_t
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[pg][g] = make_float2(0.f, 0.f);
 #pragma unroll 1
-  for (int it = 0; it < 2; ++it) {
-    const int w0 = (2 * half + it) * BITS;  // first stream word of fields 64 half + 32 it ..
-    uint32_t WA[BITS], WB[BITS];
+  for (int it = 0; it < NIT; ++it) {
+    const int w0 = 2 * half * BITS + it * WPI;  // first stream word of fields 64 half + FPI it ..
+    uint32_t WA[WPI], WB[WPI];
 #pragma unroll
-    for (int j = 0; j < BITS; ++j) {  // word w of the stream: chunk w / 4, word w % 4 of the slot's 16 bytes
+    for (int j = 0; j < WPI; ++j) {  // word w of the stream: chunk w / 4, word w % 4 of the slot's 16 bytes
       const int w = w0 + j;
       WA[j] = ra32[(16 * (w >> 2) + t) * 4 + (w & 3)];
       WB[j] = rb32[(16 * (w >> 2) + t) * 4 + (w & 3)];
     }
-    const bool tail = it == 1 && half;  // the granule's last pair is (azimuth, padding)
-    const float *qi = qh + it * 16 * G * 2;
+    const bool tail = it == NIT - 1 && half;  // the iteration's last pair is (azimuth, padding)
+    const float *qi = qh + it * PPI * G * 2;
 #pragma unroll
-    for (int pq = 0; pq < 16; ++pq) {
+    for (int pq = 0; pq < PPI; ++pq) {
       float2 uu[2];
 #pragma unroll
       for (int pg = 0; pg < 2; ++pg) {
-        const uint32_t c0 = bits_at<BITS, BITS>(pg ? WB : WA, 2 * pq * BITS);
-        const uint32_t c1 = bits_at<BITS, BITS>(pg ? WB : WA, (2 * pq + 1) * BITS);
+        const uint32_t c0 = bits_at<BITS, WPI>(pg ? WB : WA, 2 * pq * BITS);
+        const uint32_t c1 = bits_at<BITS, WPI>(pg ? WB : WA, (2 * pq + 1) * BITS);
         float2 e0, e1;
-        if (pq == 15) {
+        if (pq == PPI - 1) {
           e0 = (tail ? laz : lpol)[c0];
           const float2 t1 = lpol[c1];
           e1 = make_float2(tail ? 1.0f : t1.x, tail ? 0.0f : t1.y);
@@ -1065,22 +1069,24 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
     for (int g = 0; g < G; ++g) scg[g] = sc[g];
     const float Lh = ADA ? sc[G] : 0.f, Dh = ADA ? sc[G + 1] : 0.f;
 
-    // logits of a page (ADA from codes, dense from bf16 keys), lanes 0..15
+    // logits of a page (ADA from codes, narrow ring; dense from bf16 keys), lanes 0..15
     auto page_logits = [&](const StageMeta &mt, const uint8_t *xst, float (&l2)[G]) {
       if constexpr (ADA) {
         float f[G];
         const int ti = tier_of_bits(mt.bits);
         const float *q0 = qt + ti * Ly::QT_TIER;
         const float2 *lp = lpol + lut_off(ti), *la = laz + lut_off(ti);
-        switch (mt.bits) {
-          case 3: ada_page_f<3, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
-          case 4: ada_page_f<4, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
-          default:
-            if constexpr (!NW) {  // (the producer admits no wider page into a narrow ring)
-              if (mt.bits == 6) ada_page_f<6, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f);
-              else ada_page_f<8, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f);
-            }
-            break;
+        // (narrow ring only: the producer admits no page of b > 4 into it;
+        // the two forms below compile to faster code for their G)
+        if constexpr (G == 8) {
+          if (mt.bits == 4) ada_page_f<4, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f);
+          else ada_page_f<3, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f);
+        } else {
+          switch (mt.bits) {
+            case 3: ada_page_f<3, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
+            case 4: ada_page_f<4, G, Ly::QT_HALF>(xst, q0, lp, la, lane, f); break;
+            default: break;
+          }
         }
         const float rad = fast_exp2(fmaf((float)xst[256 * mt.bits + (lane & 15)], Dh, Lh));
 #pragma unroll
@@ -1220,42 +1226,72 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
           if (use[q]) tma_load_3d(vslot[q], &vmap, 0, mt[q].vrow, 0, vbar);
       }
       float l2[2][G];
-      bool paired = false;
-      if constexpr (ADA) {
-        paired = use[0] && use[1] && mt[0].bits == mt[1].bits && (!NW || mt[0].bits <= 4);
-      }
-      if (paired) {
-        if constexpr (ADA) {
+      if constexpr (ADA && !NW) {
+        // Wide ring (pages of every tier): one f_b call site, for a smaller
+        // instruction footprint (warps of one SM run different tiers' paths
+        // at once): a pair of one tier in one pass; otherwise each used page
+        // alone, given as both pages of its pass.
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int g = 0; g < G; ++g) l2[q][g] = 0.f;
+        const bool paired = use[0] && use[1] && mt[0].bits == mt[1].bits;
+        const int npass = paired ? 1 : 2;
+#pragma unroll 1
+        for (int pass = 0; pass < npass; ++pass) {
+          const int qa = paired ? 0 : pass, qb = paired ? 1 : pass;
+          if (!(qa ? use[1] : use[0])) continue;  // warp-uniform
           float fa[G], fb[G];
-          const int ti = tier_of_bits(mt[0].bits);
+          const int bits = qa ? mt[1].bits : mt[0].bits;
+          const int ti = tier_of_bits(bits);
           const float *q0 = qt + ti * Ly::QT_TIER;
           const float2 *lp = lpol + lut_off(ti), *la = laz + lut_off(ti);
-          if constexpr (NW) {
+          const uint8_t *ra = qa ? xst[1] : xst[0], *rb = qb ? xst[1] : xst[0];
+          switch (bits) {
+            case 4: ada_2page_f4<G, Ly::QT_HALF>(ra, rb, q0, smem_u32(lp), smem_u32(la), lane, fa, fb); break;
+            case 3: ada_2page_gen<3, G, Ly::QT_HALF>(ra, rb, q0, lp, la, lane, fa, fb); break;
+            case 6: ada_2page_gen<6, G, Ly::QT_HALF>(ra, rb, q0, lp, la, lane, fa, fb); break;
+            default: ada_2page_gen<8, G, Ly::QT_HALF>(ra, rb, q0, lp, la, lane, fa, fb); break;
+          }
+          const float rda = fast_exp2(fmaf((float)ra[256 * bits + (lane & 15)], Dh, Lh));
+          const float rdb = fast_exp2(fmaf((float)rb[256 * bits + (lane & 15)], Dh, Lh));
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float va = scg[g] * rda * fa[g], vb = scg[g] * rdb * fb[g];
+            if (qa == 0) l2[0][g] = va;
+            else l2[1][g] = va;
+            if (qb == 1) l2[1][g] = vb;
+          }
+        }
+      } else {
+        // narrow ring (b <= 4; the producer admits no wider page) and the
+        // dense path: a pair of one tier in one pass, other pages alone
+        bool paired = false;
+        if constexpr (ADA) paired = use[0] && use[1] && mt[0].bits == mt[1].bits && mt[0].bits <= 4;
+        if (paired) {
+          if constexpr (ADA) {
+            float fa[G], fb[G];
+            const int ti = tier_of_bits(mt[0].bits);
+            const float *q0 = qt + ti * Ly::QT_TIER;
+            const float2 *lp = lpol + lut_off(ti), *la = laz + lut_off(ti);
             if (mt[0].bits == 4)
               ada_2page_f4<G, Ly::QT_HALF>(xst[0], xst[1], q0, smem_u32(lp), smem_u32(la), lane, fa, fb);
             else
               ada_2page_f<3, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb);
-          } else {
-            switch (mt[0].bits) {
-              case 4: ada_2page_f4<G, Ly::QT_HALF>(xst[0], xst[1], q0, smem_u32(lp), smem_u32(la), lane, fa, fb); break;
-              case 3: ada_2page_gen<3, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb); break;
-              case 6: ada_2page_gen<6, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb); break;
-              default: ada_2page_gen<8, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb); break;
+            const int bits = mt[0].bits;
+            const float ra = fast_exp2(fmaf((float)xst[0][256 * bits + (lane & 15)], Dh, Lh));
+            const float rb = fast_exp2(fmaf((float)xst[1][256 * bits + (lane & 15)], Dh, Lh));
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              l2[0][g] = scg[g] * ra * fa[g];
+              l2[1][g] = scg[g] * rb * fb[g];
             }
           }
-          const int bits = mt[0].bits;
-          const float ra = fast_exp2(fmaf((float)xst[0][256 * bits + (lane & 15)], Dh, Lh));
-          const float rb = fast_exp2(fmaf((float)xst[1][256 * bits + (lane & 15)], Dh, Lh));
+        } else {
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            l2[0][g] = scg[g] * ra * fa[g];
-            l2[1][g] = scg[g] * rb * fb[g];
+          for (int q = 0; q < 2; ++q) {
+            if (use[q]) page_logits(mt[q], xst[q], l2[q]);  // warp-uniform
           }
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          if (use[q]) page_logits(mt[q], xst[q], l2[q]);  // warp-uniform
         }
       }
       // test the next pair's stages now (their previous phases were this

@@ -117,8 +117,9 @@ __device__ __forceinline__ uint32_t enc_record(const EncodeParams &p, const EncP
 // The 32 key rows (8 KB, contiguous) come into the warp's shared-memory
 // stage with coalesced loads (rows 264 bytes apart, so the lanes' 8-byte
 // reads of their own rows fall in different bank pairs); each lane encodes
-// its key from there (encode_key_lane); the value rows are copied one row at
-// a time by the whole warp (coalesced 256-byte reads and writes).
+// its key from there (encode_key_lane); the value rows are copied by the
+// whole warp, a row per instruction (coalesced 256-byte reads and writes),
+// eight rows in flight.
 constexpr int kEncRowStride = 264;  // bytes per staged key row
 struct EncodeSmem {
   double pol_c2[kLutEntries];
@@ -167,14 +168,24 @@ __global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const EncodePara
         encode_key_lane_bits(bits, krow, p.arena + rec, pl.slot, p.rad_lo[pl.h], p.rad_step[pl.h], sm.pol_c2,
                              sm.az_c2, p.err);
     }
-    // ---- the value rows, one row per step, the whole warp on each
+    // ---- the value rows, the whole warp on each row; eight rows' loads are
+    // issued before their stores, so their latencies overlap
     if (p.values) {
-      int64_t dst_row = go ? (((int64_t)pl.pid * p.Hkv + pl.h) * kPage + pl.slot) * kD : -1;
-      for (int j = 0; j < cnt; ++j) {
-        const int64_t dr = __shfl_sync(0xffffffffu, dst_row, j);
-        if (dr < 0) continue;  // warp-uniform
-        const uint2 v = *reinterpret_cast<const uint2 *>(p.values + (first + j) * kD + 4 * lane);
-        *reinterpret_cast<uint2 *>(p.v_pages + dr + 4 * lane) = v;
+      const int64_t dst_row = go ? (((int64_t)pl.pid * p.Hkv + pl.h) * kPage + pl.slot) * kD : -1;
+      constexpr int kRows = 8;
+      for (int j0 = 0; j0 < cnt; j0 += kRows) {
+        uint2 v[kRows];
+        int64_t dr[kRows];
+#pragma unroll
+        for (int k = 0; k < kRows; ++k) {
+          const int j = j0 + k;
+          dr[k] = __shfl_sync(0xffffffffu, dst_row, j & 31);
+          if (j >= cnt) dr[k] = -1;  // warp-uniform
+          if (dr[k] >= 0) v[k] = *reinterpret_cast<const uint2 *>(p.values + (first + j) * kD + 4 * lane);
+        }
+#pragma unroll
+        for (int k = 0; k < kRows; ++k)
+          if (dr[k] >= 0) *reinterpret_cast<uint2 *>(p.v_pages + dr[k] + 4 * lane) = v[k];
       }
     }
     __syncwarp();

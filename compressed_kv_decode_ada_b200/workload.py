@@ -5,7 +5,7 @@ from __future__ import annotations
 import torch
 
 from .cache import SpkvCache
-from .ops import encode_keys
+from .ops import encode_keys, encode_keys_packed
 from .synthetic import Workload
 
 
@@ -17,8 +17,11 @@ def build_cache(wl: Workload, device=None, with_values: bool = True) -> SpkvCach
     return cache
 
 
-def prefill(cache: SpkvCache, wl: Workload, with_values: bool = True) -> None:
-    """Encode every context token of every sequence into its page slot."""
+def prefill(cache: SpkvCache, wl: Workload, with_values: bool = True, packed: bool = True) -> None:
+    """Encode every context token of every sequence into its page slot: one
+    spkv_encode_keys call when every sequence has the same length, else one
+    spkv_encode_keys_packed call over the concatenated tokens (packed=False:
+    one spkv_encode_keys call per sequence instead)."""
     if wl.B == 0:
         return
     if len(set(int(n) for n in wl.ctx)) == 1:
@@ -29,6 +32,16 @@ def prefill(cache: SpkvCache, wl: Workload, with_values: bool = True) -> None:
         vals = wl.values.view(wl.B, n, wl.Hkv, -1) if with_values else None
         start = torch.zeros(wl.B, dtype=torch.int32, device=cache.device)
         encode_keys(cache, keys, start, wl.block_table, values=vals)
+        return
+    if packed:
+        key = ("packed_positions", str(cache.device))
+        if key not in wl.extras:  # token t of sequence s goes to position t - seq_off[s]
+            dev = cache.device
+            seq_start = torch.as_tensor(wl.seq_off.astype("int32"), device=dev)
+            dst = torch.cat([torch.arange(int(n), dtype=torch.int32, device=dev) for n in wl.ctx])
+            wl.extras[key] = (seq_start, dst)
+        seq_start, dst = wl.extras[key]
+        encode_keys_packed(cache, wl.keys, seq_start, dst, wl.block_table, values=wl.values if with_values else None)
         return
     for b in range(wl.B):
         n = int(wl.ctx[b])

@@ -116,6 +116,21 @@ def test_encode_thread_and_warp_forms_write_the_same_bytes(spkv):
     assert torch.equal(one.v_pages, steps.v_pages)
 
 
+def test_packed_and_per_sequence_prefill_write_the_same_bytes(spkv):
+    """A ragged batch prefilled by one spkv_encode_keys_packed call (the
+    default) and by one spkv_encode_keys call per sequence: identical pages."""
+    m, synthetic, workload = spkv
+    wl = synthetic.make_workload(RAGGED, device="cuda", B=5, ctx=[700, 1, 33, 2049, 160])
+    packed = m.SpkvCache(wl.num_pages, wl.Hkv, wl.page_bits, wl.rad_lo, wl.rad_step, keep_mask=wl.keep_mask)
+    perseq = m.SpkvCache(wl.num_pages, wl.Hkv, wl.page_bits, wl.rad_lo, wl.rad_step, keep_mask=wl.keep_mask)
+    workload.prefill(packed, wl)
+    workload.prefill(perseq, wl, packed=False)
+    torch.cuda.synchronize()
+    assert packed.error_flags() == 0 and perseq.error_flags() == 0
+    assert torch.equal(packed.arena, perseq.arena)
+    assert torch.equal(packed.v_pages, perseq.v_pages)
+
+
 def _last_tokens(wl):
     idx = torch.tensor([int(wl.seq_off[b]) + int(wl.ctx[b]) - 1 for b in range(wl.B)], device=wl.keys.device)
     return wl.keys[idx].contiguous(), wl.values[idx].contiguous()
