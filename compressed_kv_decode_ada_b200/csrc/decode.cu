@@ -472,11 +472,16 @@ __device__ __forceinline__ void ada_2page_f(const uint8_t *recA, const uint8_t *
 // 256-byte aligned shared address.  Each code word is spread once into
 // bytes holding 8 x code (even fields in E, odd fields in O); a field's entry
 // address is then one byte permute: the entry offset as the low byte under
-// the table's upper address bytes.
-template <int G, int QT_HALF>
+// the table's upper address bytes.  NIT = 4 or 8 shortens the body further
+// (16 or 8 fields, two words or one per page and iteration): measured faster
+// for G = 8 (NIT = 4) and in the mixed-tier kernel (NIT = 8), whose warps run
+// several tiers' paths at once; slower for G <= 4 on a b = 4 cache.
+template <int G, int QT_HALF, int NIT = 2>
 __device__ __forceinline__ void ada_2page_f4(const uint8_t *recA, const uint8_t *recB, const float *qt,
                                              uint32_t lpol_s, uint32_t laz_s, int lane, float (&fA)[G],
                                              float (&fB)[G]) {
+  static_assert(NIT == 2 || NIT == 4 || NIT == 8, "32, 16 or 8 fields per iteration");
+  constexpr int PPI = 32 / NIT, NWD = 8 / NIT;  // pairs and code words per page and iteration
   const int t = lane & 15, half = lane >> 4;
   const float *qh = qt + half * QT_HALF;
   float2 acc[2][G];
@@ -486,16 +491,30 @@ __device__ __forceinline__ void ada_2page_f4(const uint8_t *recA, const uint8_t 
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[pg][g] = make_float2(0.f, 0.f);
 #pragma unroll 1
-  for (int it = 0; it < 2; ++it) {
-    const int chunk = half * 2 + it;
-    const uint4 wa = *reinterpret_cast<const uint4 *>(recA + (chunk * 16 + t) * 16);
-    const uint4 wb = *reinterpret_cast<const uint4 *>(recB + (chunk * 16 + t) * 16);
-    const uint32_t WA[4] = {wa.x, wa.y, wa.z, wa.w}, WB[4] = {wb.x, wb.y, wb.z, wb.w};
-    // the chunk's last pair is (azimuth, padding) in the second half
-    const bool tail = it == 1 && half;
-    const float *qi = qh + it * 16 * G * 2;
+  for (int it = 0; it < NIT; ++it) {
+    uint32_t WA[NWD], WB[NWD];
+    if constexpr (NIT == 2) {
+      const int chunk = half * 2 + it;
+      const uint4 wa = *reinterpret_cast<const uint4 *>(recA + (chunk * 16 + t) * 16);
+      const uint4 wb = *reinterpret_cast<const uint4 *>(recB + (chunk * 16 + t) * 16);
+      WA[0] = wa.x; WA[1] = wa.y; WA[2] = wa.z; WA[3] = wa.w;
+      WB[0] = wb.x; WB[1] = wb.y; WB[2] = wb.z; WB[3] = wb.w;
+    } else if constexpr (NIT == 4) {  // words 2 (it & 1), +1 of chunk 2 half + it / 2
+      const int off = ((half * 2 + (it >> 1)) * 16 + t) * 16 + (it & 1) * 8;
+      const uint2 wa = *reinterpret_cast<const uint2 *>(recA + off);
+      const uint2 wb = *reinterpret_cast<const uint2 *>(recB + off);
+      WA[0] = wa.x; WA[1] = wa.y;
+      WB[0] = wb.x; WB[1] = wb.y;
+    } else {  // word it & 3 of chunk 2 half + it / 4
+      const int off = ((half * 2 + (it >> 2)) * 16 + t) * 16 + (it & 3) * 4;
+      WA[0] = *reinterpret_cast<const uint32_t *>(recA + off);
+      WB[0] = *reinterpret_cast<const uint32_t *>(recB + off);
+    }
+    // the iteration's last pair is (azimuth, padding) in the second half
+    const bool tail = it == NIT - 1 && half;
+    const float *qi = qh + it * PPI * G * 2;
 #pragma unroll
-    for (int pq = 0; pq < 16; ++pq) {
+    for (int pq = 0; pq < PPI; ++pq) {
       float2 uu[2];
 #pragma unroll
       for (int pg = 0; pg < 2; ++pg) {
@@ -503,7 +522,7 @@ __device__ __forceinline__ void ada_2page_f4(const uint8_t *recA, const uint8_t 
         const uint32_t ev = (w << 3) & 0x78787878u, od = (w >> 1) & 0x78787878u;  // CSE'd per word
         const uint32_t sel = 0x7650u | (uint32_t)(pq & 3);
         float2 e0, e1;
-        if (pq == 15) {
+        if (pq == PPI - 1) {
           e0 = lds_f2(__byte_perm(ev, tail ? laz_s : lpol_s, sel));
           const float2 t1 = lds_f2(__byte_perm(od, lpol_s, sel));
           e1 = make_float2(tail ? 1.0f : t1.x, tail ? 0.0f : t1.y);
@@ -542,18 +561,18 @@ __device__ __forceinline__ void ada_2page_f4(const uint8_t *recA, const uint8_t 
   }
 }
 
-// Pair path for any width b (used for b = 3, 6, 8; b = 4 has ada_2page_f4):
-// a rolled loop over the 64 fields of the lane's half, NIT iterations of
-// 64 / NIT fields of both pages -- 64 b / NIT bits = whole words of the
-// slot's stream, loaded per iteration -- so the loop body stays short
-// (b = 3: two iterations of 32 fields; b = 6, 8: four of 16).
+// Pair path for any width b (used for b = 3, 6, 8 in the mixed-tier kernel;
+// b = 4 has ada_2page_f4): a rolled loop over the 64 fields of the lane's
+// half, eight iterations of 8 fields of both pages -- 8 b bits of the slot's
+// stream, two words per page loaded and shifted into place per iteration --
+// so the loop body stays short (the mixed-tier kernel was bound by
+// instruction fetch: each shortening of this body measured faster).
 template <int BITS, int G, int QT_HALF>
 __device__ __forceinline__ void ada_2page_gen(const uint8_t *recA, const uint8_t *recB, const float *qt,
                                               const float2 *lpol, const float2 *laz, int lane, float (&fA)[G],
                                               float (&fB)[G]) {
-  constexpr int NIT = BITS == 3 ? 2 : 4;
-  constexpr int FPI = 64 / NIT, PPI = FPI / 2, WPI = FPI * BITS / 32;  // fields, pairs, words per iteration
-  static_assert(FPI * BITS % 32 == 0, "an iteration covers whole words");
+  constexpr int NIT = 8;
+  constexpr int FPI = 64 / NIT, PPI = FPI / 2, WPI = 2;  // fields, pairs, words per iteration
   const int t = lane & 15, half = lane >> 4;
   const float *qh = qt + half * QT_HALF;
   const uint32_t *ra32 = reinterpret_cast<const uint32_t *>(recA);
@@ -566,13 +585,21 @@ __device__ __forceinline__ void ada_2page_gen(const uint8_t *recA, const uint8_t
     for (int g = 0; g < G; ++g) acc[pg][g] = make_float2(0.f, 0.f);
 #pragma unroll 1
   for (int it = 0; it < NIT; ++it) {
-    const int w0 = 2 * half * BITS + it * WPI;  // first stream word of fields 64 half + FPI it ..
+    // word w of the stream: chunk w / 4, word w % 4 of the slot's 16 bytes
+    auto word = [&](const uint32_t *r32, int w) { return r32[(16 * (w >> 2) + t) * 4 + (w & 3)]; };
     uint32_t WA[WPI], WB[WPI];
-#pragma unroll
-    for (int j = 0; j < WPI; ++j) {  // word w of the stream: chunk w / 4, word w % 4 of the slot's 16 bytes
-      const int w = w0 + j;
-      WA[j] = ra32[(16 * (w >> 2) + t) * 4 + (w & 3)];
-      WB[j] = rb32[(16 * (w >> 2) + t) * 4 + (w & 3)];
+    {  // bits [8 b it, 8 b it + 8 b) of the half's 64 b, from two words shifted into place:
+       // sh + 8 b <= 64 (sh in {0, 8, 16, 24} for b = 3, {0, 16} for b = 6, 0 for b = 8);
+       // the second word is clamped to the slot's last (its bits are then unused)
+      static_assert(BITS == 3 || BITS == 6 || BITS == 8, "widths of the pair path");
+      const int bit0 = it * FPI * BITS, w0 = 2 * half * BITS + (bit0 >> 5), sh = bit0 & 31;
+      const int w1 = w0 + 1 < 4 * BITS ? w0 + 1 : w0;
+      const uint64_t a = ((uint64_t)word(ra32, w1) << 32 | word(ra32, w0)) >> sh;
+      const uint64_t b = ((uint64_t)word(rb32, w1) << 32 | word(rb32, w0)) >> sh;
+      WA[0] = (uint32_t)a;
+      WA[1] = (uint32_t)(a >> 32);
+      WB[0] = (uint32_t)b;
+      WB[1] = (uint32_t)(b >> 32);
     }
     const bool tail = it == NIT - 1 && half;  // the iteration's last pair is (azimuth, padding)
     const float *qi = qh + it * PPI * G * 2;
@@ -1248,7 +1275,7 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
           const float2 *lp = lpol + lut_off(ti), *la = laz + lut_off(ti);
           const uint8_t *ra = qa ? xst[1] : xst[0], *rb = qb ? xst[1] : xst[0];
           switch (bits) {
-            case 4: ada_2page_f4<G, Ly::QT_HALF>(ra, rb, q0, smem_u32(lp), smem_u32(la), lane, fa, fb); break;
+            case 4: ada_2page_f4<G, Ly::QT_HALF, 8>(ra, rb, q0, smem_u32(lp), smem_u32(la), lane, fa, fb); break;
             case 3: ada_2page_gen<3, G, Ly::QT_HALF>(ra, rb, q0, lp, la, lane, fa, fb); break;
             case 6: ada_2page_gen<6, G, Ly::QT_HALF>(ra, rb, q0, lp, la, lane, fa, fb); break;
             default: ada_2page_gen<8, G, Ly::QT_HALF>(ra, rb, q0, lp, la, lane, fa, fb); break;
@@ -1275,7 +1302,8 @@ __global__ void __launch_bounds__(Layout<ADA, G, NW>::THREADS, 2)
             const float *q0 = qt + ti * Ly::QT_TIER;
             const float2 *lp = lpol + lut_off(ti), *la = laz + lut_off(ti);
             if (mt[0].bits == 4)
-              ada_2page_f4<G, Ly::QT_HALF>(xst[0], xst[1], q0, smem_u32(lp), smem_u32(la), lane, fa, fb);
+              ada_2page_f4<G, Ly::QT_HALF, G == 8 ? 4 : 2>(xst[0], xst[1], q0, smem_u32(lp), smem_u32(la), lane, fa,
+                                                          fb);
             else
               ada_2page_f<3, G, Ly::QT_HALF>(xst[0], xst[1], q0, lp, la, lane, fa, fb);
             const int bits = mt[0].bits;
