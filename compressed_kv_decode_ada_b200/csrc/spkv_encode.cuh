@@ -25,26 +25,25 @@ namespace spkv {
 //   x > 0: the code is the largest k in [0, 2^(b-1)) with x^2 <= S c2[k]
 //          (k = 0 always: c2[0] = 1, x^2 <= S);
 //   x < 0: the code is 2^(b-1) + the largest j in [0, 2^(b-1)) with j = 0 or
-//          x^2 >= S c2[2^(b-1) + j];
+//          x^2 >= S c2[2^(b-1) + j], tested as -x^2 <= (-S) c2[2^(b-1) + j]
+//          (negation is exact, so this is the same test), which makes both
+//          halves one comparison, sx2 <= sS c2[...];
 //   x = 0: the angle is pi/2 exactly, code 2^(b-1)
 // (polar_reaches' tests, in which "x <= 0" and "x < 0" are fixed per angle;
-// c2[2^(b-1)] = 0 exactly, so k = 2^(b-1) is not reached for x > 0).
+// c2[2^(b-1)] = 0 exactly, so k = 2^(b-1) is not reached for x > 0).  The
+// test is monotone in k (true up to the code, false above), so the search
+// adds the steps 2^(b-2), ..., 1 to k while the test holds.
 template <int BITS>
 __device__ __forceinline__ int polar_code_half(double x, double S, const double *c2) {
   constexpr int H = 1 << (BITS - 1);
-  const double x2 = x * x;
   const bool pos = x > 0.0;
+  const double x2 = x * x;
+  const double sx2 = pos ? x2 : -x2, sS = pos ? S : -S;
   const double *tab = pos ? c2 : c2 + H;
-  int lo = 0, hi = H - 1;
+  int k = 0;
 #pragma unroll
-  for (int it = 0; it < BITS - 1; ++it) {
-    const int mid = (lo + hi + 1) >> 1;
-    const double rhs = S * tab[mid];
-    const bool r = pos ? x2 <= rhs : x2 >= rhs;
-    lo = r ? mid : lo;
-    hi = r ? hi : mid - 1;
-  }
-  int code = pos ? lo : H + lo;
+  for (int step = H / 2; step >= 1; step >>= 1) k = sx2 <= sS * tab[k + step] ? k + step : k;
+  int code = pos ? k : H + k;
   code = x == 0.0 ? H : code;
   return S == 0.0 ? 0 : code;
 }

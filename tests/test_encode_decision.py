@@ -9,10 +9,12 @@ section 2.1).
    cell edges, the kernel lets the sign of x_i pick the half of [0, pi] the
    polar angle lies in and searches that half's 2^(b-1) edges in b - 1 steps
    (x > 0: the largest k with x^2 <= S c2[k]; x < 0: 2^(b-1) + the largest j
-   with j = 0 or x^2 >= S c2[2^(b-1) + j]; x = 0: 2^(b-1); S = 0: 0), with
-   c2[k] = cos^2(k pi / 2^b).  Restated here and compared, code by code, with
-   the oracle's codes of random bf16 keys (equal off the cell edges) and with a
-   brute-force scan of every edge (equal everywhere, ties included).
+   with j = 0 or x^2 >= S c2[2^(b-1) + j], tested as -x^2 <= (-S) c2[...];
+   x = 0: 2^(b-1); S = 0: 0), with c2[k] = cos^2(k pi / 2^b), adding the
+   steps 2^(b-2), ..., 1 while the test holds.  Restated here and compared,
+   code by code, with the oracle's codes of random bf16 keys (equal off the
+   cell edges) and with a brute-force scan of every edge (equal everywhere,
+   ties included).
 2. The slot words.  Codes are pushed from field 127 down to 0 into a 64-bit
    accumulator (acc = acc << b | c) and word w = stream bits [32 w, 32 w + 32)
    is taken once the lowest pushed code starts at or below bit 32 w; the four
@@ -66,18 +68,20 @@ def _suffix_sums(x):
 
 
 def _polar_half(x, S, c2, b):
-    """The kernel's half-range search (restated)."""
+    """The kernel's half-range search (restated): one comparison for both
+    halves, sx2 <= sS c2[...] with the signs of x^2 and S flipped for x <= 0."""
     H = 1 << (b - 1)
-    x2 = x * x
     pos = x > 0.0
+    x2 = x * x
+    sx2, sS = (x2, S) if pos else (-x2, -S)
     tab = c2 if pos else c2[H:]
-    lo, hi = 0, H - 1
-    for _ in range(b - 1):
-        mid = (lo + hi + 1) >> 1
-        rhs = S * tab[mid]
-        r = x2 <= rhs if pos else x2 >= rhs
-        lo, hi = (mid, hi) if r else (lo, mid - 1)
-    code = lo if pos else H + lo
+    k = 0
+    step = H // 2
+    while step >= 1:
+        if sx2 <= sS * tab[k + step]:
+            k += step
+        step //= 2
+    code = k if pos else H + k
     if x == 0.0:
         code = H
     return 0 if S == 0.0 else code
