@@ -28,7 +28,9 @@ namespace spkv {
 //          x^2 >= S c2[2^(b-1) + j], tested as -x^2 <= (-S) c2[2^(b-1) + j]
 //          (negation is exact, so this is the same test), which makes both
 //          halves one comparison, sx2 <= sS c2[...];
-//   x = 0: the angle is pi/2 exactly, code 2^(b-1)
+//   x = 0: the angle is pi/2 exactly, code 2^(b-1) -- the x < 0 branch gives
+//          it: -0 <= (-S) c2[2^(b-1) + j] fails for every j >= 1 (c2 > 0
+//          there, and S c2 >= 2^-280 for bf16 inputs, so it never rounds to 0)
 // (polar_reaches' tests, in which "x <= 0" and "x < 0" are fixed per angle;
 // c2[2^(b-1)] = 0 exactly, so k = 2^(b-1) is not reached for x > 0).  The
 // test is monotone in k (true up to the code, false above), so the search
@@ -43,9 +45,7 @@ __device__ __forceinline__ int polar_code_half(double x, double S, const double 
   int k = 0;
 #pragma unroll
   for (int step = H / 2; step >= 1; step >>= 1) k = sx2 <= sS * tab[k + step] ? k + step : k;
-  int code = pos ? k : H + k;
-  code = x == 0.0 ? H : code;
-  return S == 0.0 ? 0 : code;
+  return S == 0.0 ? 0 : (pos ? k : H + k);
 }
 
 // Non-uniform quantiser (an f_b variant): polar angle a has its own edges,
@@ -71,10 +71,12 @@ __device__ __forceinline__ int polar_code_nu(double x, double S, const double *e
 }
 
 // The slot's bitstream (codes LSB first, code i at bits [i b, i b + b)) is
-// built from the top code down in a 64-bit accumulator (acc = acc << b | c),
+// built from the top group of four codes down in a 64-bit accumulator
+// (acc = acc << 4 b | grp, grp holding field i + k at bits [k b, k b + b)),
 // and word w = bits [32 w, 32 w + 32) is taken once the lowest code added
-// starts at or below bit 32 w; the four words of chunk c = w / 4 go out as one
-// 16-byte store at recp + (16 c + slot) 16 (chunk-major record layout).
+// starts at or below bit 32 w (4 b <= 32: at most one word per group, and at
+// most 32 + 4 b <= 64 bits pending); the four words of chunk c = w / 4 go out
+// as one 16-byte store at recp + (16 c + slot) 16 (chunk-major record layout).
 struct SlotWords {
   uint64_t acc = 0u;
   int w;       // next word to take (descending)
@@ -85,9 +87,9 @@ struct SlotWords {
     stage = make_uint4(0u, 0u, 0u, 0u);
   }
   template <int BITS>
-  __device__ __forceinline__ void push(int i, uint32_t c) {
-    acc = (acc << BITS) | c;
-    if (i * BITS <= 32 * w) {  // word w complete (uniform across lanes that run the same key index)
+  __device__ __forceinline__ void push_group(int i, uint32_t grp) {
+    acc = (acc << (4 * BITS)) | grp;
+    if (i * BITS <= 32 * w) {  // word w complete
       const uint32_t word = (uint32_t)(acc >> (32 * w - i * BITS));
       const int wic = w & 3;
       stage.x = wic == 0 ? word : stage.x;
@@ -134,30 +136,30 @@ __device__ __forceinline__ void encode_key_lane(const uint16_t *key, uint8_t *re
   s[1] = fma(x[1], x[1], s[2]);
   s[0] = fma(x[0], x[0], s[1]);
   double T = s[0] + 0.0;  // T_31 (T_32 = 0)
-  sw.push<BITS>(127, 0u);
-  sw.push<BITS>(126, (uint32_t)azimuth_code<BITS>(x[2], x[3], s[2] + 0.0, ac2));
-  sw.push<BITS>(125, polar(125, x[1], s[1] + 0.0));
-  sw.push<BITS>(124, polar(124, x[0], s[0] + 0.0));
-  // ---- groups 30 .. 0; each group's dims are loaded eight groups (two
-  // 32-byte sectors of the row) ahead, through a shift register
-  uint2 pf[8];
+  sw.push_group<BITS>(124, polar(124, x[0], s[0] + 0.0) | polar(125, x[1], s[1] + 0.0) << BITS |
+                               (uint32_t)azimuth_code<BITS>(x[2], x[3], s[2] + 0.0, ac2) << (2 * BITS));
+  // (field 127, the padding, is 0)
+  // ---- groups 30 .. 0; each group's dims are loaded four groups (one
+  // 32-byte sector of the row) ahead, through a shift register
+  uint2 pf[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) pf[j] = kr[30 - j];
+  for (int j = 0; j < 4; ++j) pf[j] = kr[30 - j];
 #pragma unroll 1
   for (int g = 30; g >= 0; --g) {
     bf16x4_to_f64(pf[0], x);
 #pragma unroll
-    for (int j = 0; j < 7; ++j) pf[j] = pf[j + 1];
-    pf[7] = g >= 8 ? kr[g - 8] : make_uint2(0u, 0u);
+    for (int j = 0; j < 3; ++j) pf[j] = pf[j + 1];
+    pf[3] = g >= 4 ? kr[g - 4] : make_uint2(0u, 0u);
     s[3] = x[3] * x[3];
     s[2] = fma(x[2], x[2], s[3]);
     s[1] = fma(x[1], x[1], s[2]);
     s[0] = fma(x[0], x[0], s[1]);
     const double Tn = T;  // T_(g+1)
     T = s[0] + Tn;        // T_g
+    uint32_t grp = 0u;
 #pragma unroll
-    for (int k = 3; k >= 0; --k)
-      sw.push<BITS>(4 * g + k, polar(4 * g + k, x[k], s[k] + Tn));
+    for (int k = 3; k >= 0; --k) grp |= polar(4 * g + k, x[k], s[k] + Tn) << (k * BITS);
+    sw.push_group<BITS>(4 * g, grp);
   }
   // ---- radius code from S_0 = T_0 = ||k||^2
   int c = 0;

@@ -10,15 +10,16 @@ section 2.1).
    polar angle lies in and searches that half's 2^(b-1) edges in b - 1 steps
    (x > 0: the largest k with x^2 <= S c2[k]; x < 0: 2^(b-1) + the largest j
    with j = 0 or x^2 >= S c2[2^(b-1) + j], tested as -x^2 <= (-S) c2[...];
-   x = 0: 2^(b-1); S = 0: 0), with c2[k] = cos^2(k pi / 2^b), adding the
-   steps 2^(b-2), ..., 1 while the test holds.  Restated here and compared,
-   code by code, with the oracle's codes of random bf16 keys (equal off the
-   cell edges) and with a brute-force scan of every edge (equal everywhere,
-   ties included).
-2. The slot words.  Codes are pushed from field 127 down to 0 into a 64-bit
-   accumulator (acc = acc << b | c) and word w = stream bits [32 w, 32 w + 32)
-   is taken once the lowest pushed code starts at or below bit 32 w; the four
-   words of chunk w / 4 land at byte (16 (w / 4) + slot) 16 of the record.
+   x = 0: 2^(b-1), which the x < 0 branch gives; S = 0: 0), with
+   c2[k] = cos^2(k pi / 2^b), adding the steps 2^(b-2), ..., 1 while the test
+   holds.  Restated here and compared, code by code, with the oracle's codes
+   of random bf16 keys (equal off the cell edges) and with a brute-force scan
+   of every edge (equal everywhere, ties included).
+2. The slot words.  Codes are pushed four at a time (fields 4g .. 4g + 3,
+   groups 31 down to 0) into a 64-bit accumulator (acc = acc << 4b | grp) and
+   word w = stream bits [32 w, 32 w + 32) is taken once the lowest pushed code
+   starts at or below bit 32 w; the four words of chunk w / 4 land at byte
+   (16 (w / 4) + slot) 16 of the record.
    Restated here, and the record read back with the layout reader the GPU
    parity tests use (the chunk-major layout of the library header).
 
@@ -81,10 +82,7 @@ def _polar_half(x, S, c2, b):
         if sx2 <= sS * tab[k + step]:
             k += step
         step //= 2
-    code = k if pos else H + k
-    if x == 0.0:
-        code = H
-    return 0 if S == 0.0 else code
+    return 0 if S == 0.0 else (k if pos else H + k)
 
 
 def _polar_scan(x, S, c2, b):
@@ -161,9 +159,13 @@ def _slot_words(codes, b, slot, rec):
     acc, w = 0, nwords - 1
     stage = [0, 0, 0, 0]
     mask64 = (1 << 64) - 1
-    for i in range(127, -1, -1):
-        c = int(codes[i]) if i < 127 else 0
-        acc = ((acc << b) | c) & mask64
+    for g in range(31, -1, -1):
+        grp = 0
+        for k in range(4):
+            i = 4 * g + k
+            grp |= (int(codes[i]) if i < 127 else 0) << (k * b)
+        acc = ((acc << (4 * b)) | grp) & mask64
+        i = 4 * g
         if i * b <= 32 * w:
             word = (acc >> (32 * w - i * b)) & 0xFFFFFFFF
             stage[w & 3] = word
