@@ -139,17 +139,16 @@ __device__ __forceinline__ void encode_key_lane(const uint16_t *key, uint8_t *re
   sw.push_group<BITS>(124, polar(124, x[0], s[0] + 0.0) | polar(125, x[1], s[1] + 0.0) << BITS |
                                (uint32_t)azimuth_code<BITS>(x[2], x[3], s[2] + 0.0, ac2) << (2 * BITS));
   // (field 127, the padding, is 0)
-  // ---- groups 30 .. 0; each group's dims are loaded four groups (one
-  // 32-byte sector of the row) ahead, through a shift register
-  uint2 pf[4];
+  // ---- groups 30 .. 0; each group's dims are loaded two groups ahead,
+  // through a shift register
+  uint2 pf[2];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) pf[j] = kr[30 - j];
+  for (int j = 0; j < 2; ++j) pf[j] = kr[30 - j];
 #pragma unroll 1
   for (int g = 30; g >= 0; --g) {
     bf16x4_to_f64(pf[0], x);
-#pragma unroll
-    for (int j = 0; j < 3; ++j) pf[j] = pf[j + 1];
-    pf[3] = g >= 4 ? kr[g - 4] : make_uint2(0u, 0u);
+    pf[0] = pf[1];
+    pf[1] = g >= 2 ? kr[g - 2] : make_uint2(0u, 0u);
     s[3] = x[3] * x[3];
     s[2] = fma(x[2], x[2], s[3]);
     s[1] = fma(x[1], x[1], s[2]);
