@@ -130,7 +130,7 @@ struct EncodeSmem {
 __global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const EncodeParams p) {
   extern __shared__ __align__(16) uint8_t enc_smem_raw[];
   EncodeSmem &sm = *reinterpret_cast<EncodeSmem *>(enc_smem_raw);
-  build_edge_tables(sm.pol_c2, sm.az_c2, threadIdx.x, kEncThreads);
+  build_edge_tables(sm.pol_c2, sm.az_c2, threadIdx.x, kEncThreads, true);
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   uint8_t *stage = sm.rows[wid];
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const EncodePara
 // the same arithmetic (encode_key_warp_seq), so no thread runs a whole key.
 __global__ void __launch_bounds__(kEncThreads) encode_kernel_warp(const EncodeParams p) {
   __shared__ double pol_c2[kLutEntries], az_c2[kLutEntries];
-  build_edge_tables(pol_c2, az_c2, threadIdx.x, kEncThreads);
+  build_edge_tables(pol_c2, az_c2, threadIdx.x, kEncThreads, true);
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (kEncThreads / 32) + (threadIdx.x >> 5);
@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel_warp(const EncodePa
     if (lane == 0) set_err(p.err, st);
     return;
   }
-  encode_key_warp_seq_bits(bits, p.keys + item * kD, p.arena + rec, pl.slot, p.rad_lo[pl.h], p.rad_step[pl.h],
+  encode_key_warp_seq_bits<true>(bits, p.keys + item * kD, p.arena + rec, pl.slot, p.rad_lo[pl.h], p.rad_step[pl.h],
                            pol_c2, az_c2, lane, p.err);
   if (p.values) {
     const uint2 v = *reinterpret_cast<const uint2 *>(p.values + item * kD + 4 * lane);

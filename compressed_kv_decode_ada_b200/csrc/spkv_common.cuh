@@ -322,11 +322,16 @@ __device__ __forceinline__ int find_seq(const int32_t *P, int B, int64_t u) {
 // Computed as (1 + cos 2 theta) / 2 so that the edges at multiples of pi/4,
 // the only ones a bf16 input can hit exactly, get the exact values 1, 1/2, 0:
 // an exact tie is then decided exactly (to the upper cell).
-__device__ __forceinline__ void build_edge_tables(double *pol_c2, double *az_c2, int tid, int nthreads) {
+// half_signed: the polar entries of the lower half of [0, pi] (k < 2^(b-1))
+// as above and those of the upper half negated, -cos^2 (the bulk encoder's
+// one-comparison search, polar_code_half<BITS, true>).
+__device__ __forceinline__ void build_edge_tables(double *pol_c2, double *az_c2, int tid, int nthreads,
+                                                  bool half_signed = false) {
   for (int i = tid; i < kLutEntries; i += nthreads) {
     const int t = i < 8 ? 0 : i < 24 ? 1 : i < 88 ? 2 : 3;
     const int b = bits_of_tier(t), k = i - lut_off(t);
-    pol_c2[i] = 0.5 * (1.0 + cospi((double)(2 * k) / (double)(1 << b)));
+    const double c2 = 0.5 * (1.0 + cospi((double)(2 * k) / (double)(1 << b)));
+    pol_c2[i] = half_signed && 2 * k >= (1 << b) ? -c2 : c2;
     az_c2[i] = 0.5 * (1.0 + cospi((double)(4 * k) / (double)(1 << b)));
   }
 }

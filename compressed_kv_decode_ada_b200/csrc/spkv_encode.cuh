@@ -25,27 +25,31 @@ namespace spkv {
 //   x > 0: the code is the largest k in [0, 2^(b-1)) with x^2 <= S c2[k]
 //          (k = 0 always: c2[0] = 1, x^2 <= S);
 //   x < 0: the code is 2^(b-1) + the largest j in [0, 2^(b-1)) with j = 0 or
-//          x^2 >= S c2[2^(b-1) + j], tested as -x^2 <= (-S) c2[2^(b-1) + j]
-//          (negation is exact, so this is the same test), which makes both
-//          halves one comparison, sx2 <= sS c2[...];
+//          x^2 >= S c2[2^(b-1) + j], tested as -x^2 <= S (-c2[2^(b-1) + j])
+//          (negation is exact, so this is the same test);
 //   x = 0: the angle is pi/2 exactly, code 2^(b-1) -- the x < 0 branch gives
-//          it: -0 <= (-S) c2[2^(b-1) + j] fails for every j >= 1 (c2 > 0
+//          it: -0 <= -S c2[2^(b-1) + j] fails for every j >= 1 (c2 > 0
 //          there, and S c2 >= 2^-280 for bf16 inputs, so it never rounds to 0)
 // (polar_reaches' tests, in which "x <= 0" and "x < 0" are fixed per angle;
 // c2[2^(b-1)] = 0 exactly, so k = 2^(b-1) is not reached for x > 0).  The
-// test is monotone in k (true up to the code, false above), so the search
-// adds the steps 2^(b-2), ..., 1 to k while the test holds.
-template <int BITS>
+// test is monotone (true up to the code, false above), so the search adds the
+// steps 2^(b-2), ..., 1 to the code while the test holds, starting from 0
+// (x > 0) or 2^(b-1) (x <= 0): one fp64 product and one comparison per step,
+// sx2 <= S e[k] with sx2 = x |x| (exactly x^2 or -x^2).
+//   HS (half-signed table, build_edge_tables(..., true)): e[k] = c2[k] below
+//       2^(b-1) and -c2[k] from 2^(b-1) on;
+//   !HS (the plain table): e[k] = c2[k], and the sign goes on S instead,
+//       sx2 <= (-S) c2[k] for x <= 0 (the same products, negated exactly).
+template <int BITS, bool HS = false>
 __device__ __forceinline__ int polar_code_half(double x, double S, const double *c2) {
   constexpr int H = 1 << (BITS - 1);
   const bool pos = x > 0.0;
-  const double x2 = x * x;
-  const double sx2 = pos ? x2 : -x2, sS = pos ? S : -S;
-  const double *tab = pos ? c2 : c2 + H;
-  int k = 0;
+  const double sx2 = x * fabs(x);
+  const double sS = HS || pos ? S : -S;
+  int k = pos ? 0 : H;
 #pragma unroll
-  for (int step = H / 2; step >= 1; step >>= 1) k = sx2 <= sS * tab[k + step] ? k + step : k;
-  return S == 0.0 ? 0 : (pos ? k : H + k);
+  for (int step = H / 2; step >= 1; step >>= 1) k = sx2 <= sS * c2[k + step] ? k + step : k;
+  return S == 0.0 ? 0 : k;
 }
 
 // Non-uniform quantiser (an f_b variant): polar angle a has its own edges,
@@ -124,7 +128,7 @@ __device__ __forceinline__ void encode_key_lane(const uint16_t *key, uint8_t *re
   constexpr int NE = (1 << BITS) - 1;
   auto polar = [&](int a, double x, double S) -> uint32_t {
     if constexpr (NU) return (uint32_t)polar_code_nu<BITS>(x, S, nu_ec + a * NE);
-    else return (uint32_t)polar_code_half<BITS>(x, S, pc2);
+    else return (uint32_t)polar_code_half<BITS, true>(x, S, pc2);
   };
   SlotWords sw(recp, slot, 4 * BITS);
   const uint2 *kr = reinterpret_cast<const uint2 *>(key);
@@ -205,7 +209,7 @@ __device__ __forceinline__ void encode_key_lane_nu_bits(int bits, const uint16_t
 // runs down the lanes one addition at a time (the same additions, so the
 // same roundings); each lane decides its four codes, and the slot's words are
 // put together by funnel shifts across lanes.
-template <int BITS>
+template <int BITS, bool HS>
 __device__ __forceinline__ void encode_key_warp_seq(const uint16_t *key, uint8_t *recp, int slot, float Lf,
                                                     float Df, const double *pc2, const double *ac2, int lane,
                                                     uint32_t *err) {
@@ -229,7 +233,7 @@ __device__ __forceinline__ void encode_key_warp_seq(const uint16_t *key, uint8_t
   for (int k = 0; k < 4; ++k) {
     const int a = 4 * lane + k;
     const double S = s[k] + Tn;
-    int c = polar_code_half<BITS>(x[k], S, pc2);
+    int c = polar_code_half<BITS, HS>(x[k], S, pc2);
     if (a >= 126) c = a == 126 ? azimuth_code<BITS>(x[2], x[3], S, ac2) : 0;
     grp |= (uint32_t)c << (k * BITS);
   }
@@ -261,17 +265,19 @@ __device__ __forceinline__ void encode_key_warp_seq(const uint16_t *key, uint8_t
   __syncwarp();
 }
 
-// encode_key_warp_seq for the tier of `bits` (a valid tier).
+// encode_key_warp_seq for the tier of `bits` (a valid tier); HS: pol_c2 is
+// the half-signed table (build_edge_tables(..., true)).
+template <bool HS = false>
 __device__ __forceinline__ void encode_key_warp_seq_bits(int bits, const uint16_t *key, uint8_t *recp, int slot,
                                                          float Lf, float Df, const double *pol_c2,
                                                          const double *az_c2, int lane, uint32_t *err) {
   const int t = tier_of_bits(bits);
   const double *pc2 = pol_c2 + lut_off(t), *ac2 = az_c2 + lut_off(t);
   switch (bits) {
-    case 3: encode_key_warp_seq<3>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
-    case 4: encode_key_warp_seq<4>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
-    case 6: encode_key_warp_seq<6>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
-    default: encode_key_warp_seq<8>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
+    case 3: encode_key_warp_seq<3, HS>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
+    case 4: encode_key_warp_seq<4, HS>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
+    case 6: encode_key_warp_seq<6, HS>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
+    default: encode_key_warp_seq<8, HS>(key, recp, slot, Lf, Df, pc2, ac2, lane, err); break;
   }
 }
 

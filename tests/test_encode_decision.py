@@ -9,10 +9,11 @@ section 2.1).
    cell edges, the kernel lets the sign of x_i pick the half of [0, pi] the
    polar angle lies in and searches that half's 2^(b-1) edges in b - 1 steps
    (x > 0: the largest k with x^2 <= S c2[k]; x < 0: 2^(b-1) + the largest j
-   with j = 0 or x^2 >= S c2[2^(b-1) + j], tested as -x^2 <= (-S) c2[...];
+   with j = 0 or x^2 >= S c2[2^(b-1) + j], tested as -x^2 <= S (-c2[...]);
    x = 0: 2^(b-1), which the x < 0 branch gives; S = 0: 0), with
    c2[k] = cos^2(k pi / 2^b), adding the steps 2^(b-2), ..., 1 while the test
-   holds.  Restated here and compared, code by code, with the oracle's codes
+   holds; the bulk encoder keeps -c2 in the table's upper half, the decode's
+   fused append puts the sign on S (both restated).  Restated here and compared, code by code, with the oracle's codes
    of random bf16 keys (equal off the cell edges) and with a brute-force scan
    of every edge (equal everywhere, ties included).
 2. The slot words.  Codes are pushed four at a time (fields 4g .. 4g + 3,
@@ -68,21 +69,27 @@ def _suffix_sums(x):
     return S
 
 
-def _polar_half(x, S, c2, b):
-    """The kernel's half-range search (restated): one comparison for both
-    halves, sx2 <= sS c2[...] with the signs of x^2 and S flipped for x <= 0."""
+def _polar_half(x, S, c2, b, half_signed=True):
+    """The kernel's half-range search (restated): the code starts at 0 (x > 0)
+    or 2^(b-1) (x <= 0) and takes the steps 2^(b-2) .. 1 while
+    x |x| <= S e[k]; e is the half-signed table (-c2 from 2^(b-1) on), or the
+    plain one with the sign on S instead (the decode's fused append)."""
     H = 1 << (b - 1)
     pos = x > 0.0
-    x2 = x * x
-    sx2, sS = (x2, S) if pos else (-x2, -S)
-    tab = c2 if pos else c2[H:]
-    k = 0
+    sx2 = x * abs(x)
+    if half_signed:
+        e = np.where(np.arange(1 << b) >= H, -c2, c2)
+        sS = S
+    else:
+        e = c2
+        sS = S if pos else -S
+    k = 0 if pos else H
     step = H // 2
     while step >= 1:
-        if sx2 <= sS * tab[k + step]:
+        if sx2 <= sS * e[k + step]:
             k += step
         step //= 2
-    return 0 if S == 0.0 else (k if pos else H + k)
+    return 0 if S == 0.0 else k
 
 
 def _polar_scan(x, S, c2, b):
@@ -127,6 +134,7 @@ def test_half_range_search_matches_the_oracle_codes(b):
         S = _suffix_sums(x)
         for i in range(126):
             got = _polar_half(x[i], S[i], c2, b)
+            assert got == _polar_half(x[i], S[i], c2, b, half_signed=False)
             assert got == _polar_scan(x[i], S[i], c2, b), (t, i, x[i], S[i])
             if not edge[t, i]:
                 assert got == codes[t, i], (t, i, got, codes[t, i], apos[t, i])
@@ -147,8 +155,9 @@ def test_half_range_search_on_exact_edges(b):
     assert _polar_half(3.0, 9.0, c2, b) == 0
     assert _polar_half(-3.0, 9.0, c2, b) == n - 1  # phi = pi: clamped to the last cell
     assert _polar_half(0.0, 0.0, c2, b) == 0
-    for x, S in [(1.0, 2.0), (0.0, 5.0), (-1.0, 2.0), (3.0, 9.0), (-3.0, 9.0)]:
+    for x, S in [(1.0, 2.0), (0.0, 5.0), (-0.0, 5.0), (-1.0, 2.0), (3.0, 9.0), (-3.0, 9.0)]:
         assert _polar_half(x, S, c2, b) == _polar_scan(x, S, c2, b)
+        assert _polar_half(x, S, c2, b, half_signed=False) == _polar_scan(x, S, c2, b)
         phi = math.atan2(math.sqrt(max(S - x * x, 0.0)), x)
         assert _polar_half(x, S, c2, b) == oracle.angle_code(phi, b, False)
 
