@@ -40,16 +40,28 @@ namespace spkv {
 //       2^(b-1) and -c2[k] from 2^(b-1) on;
 //   !HS (the plain table): e[k] = c2[k], and the sign goes on S instead,
 //       sx2 <= (-S) c2[k] for x <= 0 (the same products, negated exactly).
+// An fp64 load from a 32-bit shared-window address (the edge tables are
+// written before the barrier that precedes every search).
+__device__ __forceinline__ double lds_f64(uint32_t addr) {
+  double v;
+  asm volatile("ld.shared.f64 %0, [%1];" : "=d"(v) : "r"(addr));
+  return v;
+}
+
 template <int BITS, bool HS = false>
 __device__ __forceinline__ int polar_code_half(double x, double S, const double *c2) {
   constexpr int H = 1 << (BITS - 1);
   const bool pos = x > 0.0;
   const double sx2 = x * fabs(x);
   const double sS = HS || pos ? S : -S;
-  int k = pos ? 0 : H;
+  const uint32_t base = smem_u32(c2);
+  uint32_t a = pos ? base : base + 8u * H;  // the entry of the code so far
 #pragma unroll
-  for (int step = H / 2; step >= 1; step >>= 1) k = sx2 <= sS * c2[k + step] ? k + step : k;
-  return S == 0.0 ? 0 : k;
+  for (int step = H / 2; step >= 1; step >>= 1) {
+    const uint32_t an = a + 8u * step;
+    a = sx2 <= sS * lds_f64(an) ? an : a;
+  }
+  return S == 0.0 ? 0 : (int)((a - base) >> 3);
 }
 
 // Non-uniform quantiser (an f_b variant): polar angle a has its own edges,
