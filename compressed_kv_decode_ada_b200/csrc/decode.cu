@@ -293,6 +293,15 @@ __device__ __forceinline__ uint32_t bits_at(const uint32_t (&W)[NW], int bit) {
   else v = __funnelshift_r(W[w], W[w + 1], sh);
   return v & ((1u << NB) - 1u);
 }
+// 8 x (NB bits of the lane's code words starting at bit `bit`): the byte
+// offset of the code's float2 table entry, one shift and one mask.
+template <int NB, int NW>
+__device__ __forceinline__ uint32_t off8_at(const uint32_t (&W)[NW], int bit) {
+  const int w = bit >> 5, sh = bit & 31;
+  constexpr uint32_t m = ((1u << NB) - 1u) << 3;
+  if (sh + NB <= 32) return (sh >= 3 ? W[w] >> (sh - 3) : W[w] << (3 - sh)) & m;
+  return __funnelshift_r(W[w], W[w + 1], sh - 3) & m;  // (sh > 32 - NB >= 24: sh - 3 >= 0)
+}
 template <int BITS>
 __device__ __forceinline__ uint32_t code_at(const uint32_t (&W)[2 * BITS], int a) {
   return bits_at<BITS, 2 * BITS>(W, a * BITS);
@@ -573,6 +582,7 @@ __device__ __forceinline__ void ada_2page_gen(const uint8_t *recA, const uint8_t
                                               float (&fB)[G]) {
   constexpr int NIT = 8;
   constexpr int FPI = 64 / NIT, PPI = FPI / 2, WPI = 2;  // fields, pairs, words per iteration
+  const uint32_t lpol_s = smem_u32(lpol), laz_s = smem_u32(laz);
   const int t = lane & 15, half = lane >> 4;
   const float *qh = qt + half * QT_HALF;
   const uint32_t *ra32 = reinterpret_cast<const uint32_t *>(recA);
@@ -608,16 +618,16 @@ __device__ __forceinline__ void ada_2page_gen(const uint8_t *recA, const uint8_t
       float2 uu[2];
 #pragma unroll
       for (int pg = 0; pg < 2; ++pg) {
-        const uint32_t c0 = bits_at<BITS, WPI>(pg ? WB : WA, 2 * pq * BITS);
-        const uint32_t c1 = bits_at<BITS, WPI>(pg ? WB : WA, (2 * pq + 1) * BITS);
+        const uint32_t o0 = off8_at<BITS, WPI>(pg ? WB : WA, 2 * pq * BITS);
+        const uint32_t o1 = off8_at<BITS, WPI>(pg ? WB : WA, (2 * pq + 1) * BITS);
         float2 e0, e1;
         if (pq == PPI - 1) {
-          e0 = (tail ? laz : lpol)[c0];
-          const float2 t1 = lpol[c1];
+          e0 = lds_f2((tail ? laz_s : lpol_s) + o0);
+          const float2 t1 = lds_f2(lpol_s + o1);
           e1 = make_float2(tail ? 1.0f : t1.x, tail ? 0.0f : t1.y);
         } else {
-          e0 = lpol[c0];
-          e1 = lpol[c1];
+          e0 = lds_f2(lpol_s + o0);
+          e1 = lds_f2(lpol_s + o1);
         }
         const float u0 = Ps[pg] * e0.x, tt = Ps[pg] * e0.y;
         uu[pg] = make_float2(u0, tt * e1.x);
