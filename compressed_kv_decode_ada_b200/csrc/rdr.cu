@@ -92,7 +92,8 @@ __device__ __forceinline__ double bf16_abs_f64(uint32_t h16) {
 }
 
 // One warp per tile of tok_per_tile tokens (tok_per_tile * Hkv <= 32 key
-// rows): a coalesced copy of the tile's rows into shared memory (rows padded
+// rows): a coalesced copy of the tile's rows into shared memory (16-byte
+// asynchronous copies, all sixteen of a lane in flight at once; rows padded
 // to 272 bytes, so that the row-per-lane reads below are conflict-free), then
 // lane r sums the squares of row r in ascending order (each square of a bf16
 // value is exact in fp64, so n2 + x * x rounded once, an FMA, is the sum of
@@ -121,21 +122,16 @@ __global__ void __launch_bounds__(kWThreads, 6) rdr_weights_kernel(const WeightP
     const int rows = ntok * p.Hkv;
     const int nchunks = rows * kRowU4;
     const uint4 *src = reinterpret_cast<const uint4 *>(p.keys) + t0 * p.Hkv * kRowU4;
-    // the tile in two rounds of 8 chunks per lane (registers stay under 64)
+    // the tile: 16 asynchronous 16-byte copies per lane, all in flight at once
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      uint4 v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int c = lane + 32 * (8 * r + i);
-        if (c < nchunks) v[i] = __ldcs(src + c);  // streamed once: evict-first
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int c = lane + 32 * (8 * r + i);
-        if (c < nchunks) tl[(c >> 4) * kTileU4 + (c & 15)] = v[i];
-      }
+    for (int i = 0; i < 16; ++i) {
+      const int c = lane + 32 * i;
+      if (c < nchunks)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(tl + (c >> 4) * kTileU4 + (c & 15))),
+                     "l"(src + c)
+                     : "memory");
     }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
     __syncwarp();
     double pr = 0.0;  // qn_h * ||k_{t,h}|| of this lane's row
     const int h = lane % p.Hkv;
