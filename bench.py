@@ -362,6 +362,44 @@ def compare_paths(args, spkv, workload, wl, cache, ctx, max_ctx, splits, ws, str
     res["encode_unit"] = "(token, kv head) keys/s, with values"
     res["resident_bytes_per_token"] = {"ada": cache.resident_bytes() / tokens,
                                        "dense_bf16": 2 * wl.Hkv * 256.0}
+    # f_b variants of the same batch: the exact (unquantised) unit query, and
+    # the non-uniform angle quantiser at b = 4 (its own cache of the batch)
+    exq_ms = timeit(lambda: spkv.decode_attention(cache, wl.q, wl.block_table, ctx, max_ctx, ws=ws,
+                                                  num_splits=splits, stream=stream, exact_q=True))
+    res["exact_q_decode_ms"] = exq_ms
+    if len(set(int(c) for c in wl.ctx)) == 1:
+        ec, mc, msn = (torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in spkv.nonuniform_tables(128, 4))
+        nu = spkv.SpkvCache(wl.num_pages, wl.Hkv, np.full(wl.num_pages, 4, np.int64), wl.rad_lo, wl.rad_step,
+                            device=dev, keep_mask=wl.keep_mask)
+        n0 = int(wl.ctx[0])
+        kv, vv = wl.keys.view(wl.B, n0, wl.Hkv, -1), wl.values.view(wl.B, n0, wl.Hkv, -1)
+        zero = torch.zeros(wl.B, dtype=torch.int32, device=dev)
+        nu_enc = timeit(lambda: spkv.encode_keys_nonuniform(nu, kv, zero, wl.block_table, 4, ec, values=vv,
+                                                            stream=stream))
+        nu_dec = timeit(lambda: spkv.decode_attention_nonuniform(nu, wl.q, wl.block_table, ctx, max_ctx, 4, ec, mc,
+                                                                 msn, stream=stream))
+        if nu.error_flags():
+            raise RuntimeError(f"non-uniform cache: device error flags {nu.error_flags():#x}")
+        res["nonuniform_b4"] = {"encode_ms": nu_enc, "encode_keys_per_s": tokens * wl.Hkv / (nu_enc * 1e-3),
+                                "decode_ms": nu_dec, "decode_kv_tokens_per_s": tokens / (nu_dec * 1e-3)}
+        del nu
+    # the page-sharded form of the step on one GPU: two shards' partial
+    # decodes (each a contiguous half of every sequence's pages) and the merge
+    # of their records -- the kernels of a two-GPU step, run in sequence
+    from compressed_kv_decode_ada_b200 import sharded
+
+    shards = []
+    for r in range(2):
+        bt, lc = sharded.shard_batch(wl.block_table_np, wl.ctx, 2, r)
+        shards.append((torch.as_tensor(bt, device=dev), torch.as_tensor(lc, device=dev), int(lc.max())))
+    parts = torch.empty((2, wl.B, wl.Hq, 132), dtype=torch.float32, device=dev)
+
+    def two_shards():
+        for r, (bt, lc, mc_) in enumerate(shards):
+            spkv.decode_attention_partial(cache, wl.q, bt, lc, mc_, partial=parts[r], ws=ws, stream=stream)
+        spkv.merge_partials(parts, stream=stream)
+
+    res["sharded_2_on_1gpu_ms"] = timeit(two_shards)
     # RDR controller (weights kernel + one cluster per sequence) over the
     # batch's context keys: 35% of the b = 8 bytes, sinks + last 64 protected
     ri = synthetic.make_rdr_inputs(wl, budget_frac=0.35)

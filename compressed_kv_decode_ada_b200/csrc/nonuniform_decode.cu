@@ -122,6 +122,11 @@ __global__ void __launch_bounds__(kNuThreads) nu_decode_kernel(const NuParams p)
   __shared__ uint8_t qcodes[G][128];
   __shared__ float wm[kNuWarps][G], wl[kNuWarps][G];
   __shared__ float wacc[kNuWarps][G][128];
+  // b <= 4: the (cos, sin) table in shared memory (one angle's 2^b entries
+  // are one 64- or 128-byte row, so a warp's lookups of one angle never
+  // conflict); wider tables are read through L1
+  constexpr bool kSmemTab = BITS <= 4;
+  __shared__ float2 stab[kSmemTab ? 127 * N : 1];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int row = blockIdx.x / p.S, split = blockIdx.x - row * p.S;
   const int b = row / p.Hkv, h = row - b * p.Hkv;
@@ -135,6 +140,8 @@ __global__ void __launch_bounds__(kNuThreads) nu_decode_kernel(const NuParams p)
   const int t_begin = pg0 * kPage, t_end = min(pg1 * kPage, ctx);
 
   build_edge_tables(pol_c2, az_c2, tid, kNuThreads);
+  if constexpr (kSmemTab)
+    for (int i = tid; i < 127 * N; i += kNuThreads) stab[i] = __ldg(p.tab + i);
   __syncthreads();
   if (tid < G) {  // the query heads' codes and scales (log2 units)
     const double n2 = nu_query_codes<BITS>(p.q + ((int64_t)b * p.Hq + h * G + tid) * kD, p.ec,
@@ -196,7 +203,10 @@ __global__ void __launch_bounds__(kNuThreads) nu_decode_kernel(const NuParams p)
       float P = 1.0f;
 #pragma unroll
       for (int j = 0; j < 127; ++j) {
-        const float2 cs = __ldg(&p.tab[j * N + nu_code<BITS>(wv, j)]);
+        const int e = j * N + (int)nu_code<BITS>(wv, j);
+        float2 cs;
+        if constexpr (kSmemTab) cs = stab[e];
+        else cs = __ldg(p.tab + e);
         const float u = P * cs.x;
         P *= cs.y;
 #pragma unroll
@@ -284,14 +294,16 @@ __global__ void __launch_bounds__(kNuThreads) nu_decode_kernel(const NuParams p)
   }
 }
 
-// Splits per (sequence, kv head) row: explicit, or about two CTAs per SM in
-// all, at most one per page.  0 on a device error.
+// Splits per (sequence, kv head) row: explicit, or about kNuCtasPerSM CTAs
+// per SM in all (the CTA is small: several per SM keep its latency-bound
+// token loop fed), at most one per page.  0 on a device error.
+constexpr int kNuCtasPerSM = 6;
 int nu_splits(int B, int Hkv, int max_ctx, int num_splits) {
   if (num_splits > 0) return num_splits;
   const int sms = device_sm_count();
   if (sms <= 0) return 0;
   const int64_t rows = (int64_t)B * Hkv;
-  int64_t S = rows > 0 ? (2 * (int64_t)sms + rows - 1) / rows : 1;
+  int64_t S = rows > 0 ? (kNuCtasPerSM * (int64_t)sms + rows - 1) / rows : 1;
   const int64_t pages = ((int64_t)max_ctx + kPage - 1) / kPage;
   if (S > pages) S = pages;
   return (int)(S < 1 ? 1 : S);
