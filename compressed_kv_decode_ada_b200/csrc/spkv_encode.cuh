@@ -67,23 +67,23 @@ __device__ __forceinline__ int polar_code_half(double x, double S, const double 
 // Non-uniform quantiser (an f_b variant): polar angle a has its own edges,
 // ec[j - 1] = cos theta_j (j = 1 .. 2^b - 1, increasing angles), and its code
 // is the largest j whose edge it reaches (j = 0 always), by the same exact
-// test: phi >= theta <=> x <= sqrt(S) cos theta, decided on x^2 vs S cos^2
-// and the signs.
+// test: phi >= theta <=> x <= sqrt(S) cos theta.  With signed squares it is
+// one comparison for either sign of cos theta:
+//   x |x| <= S (c |c|)   (c = cos theta)
+// -- for c >= 0 it holds iff x <= 0 or x^2 <= S c^2, for c < 0 iff x < 0 and
+// x^2 >= S c^2 (S c^2 > 0 there), which is the test; c |c| and x |x| are the
+// rounded squares with a sign, so the products round as S (c c) does.  The
+// search adds the steps 2^(b-1), ..., 1 while the test holds.
 template <int BITS>
 __device__ __forceinline__ int polar_code_nu(double x, double S, const double *ec) {
-  if (S == 0.0) return 0;
-  const double x2 = x * x;
-  int lo = 0, hi = (1 << BITS) - 1;
+  const double sx2 = x * fabs(x);
+  int k = 0;
 #pragma unroll
-  for (int it = 0; it < BITS; ++it) {
-    const int mid = (lo + hi + 1) >> 1;
-    const double c = ec[mid - 1];
-    const double rhs = S * (c * c);
-    const bool r = c >= 0.0 ? (x <= 0.0 || x2 <= rhs) : (x < 0.0 && x2 >= rhs);
-    lo = r ? mid : lo;
-    hi = r ? hi : mid - 1;
+  for (int step = 1 << (BITS - 1); step >= 1; step >>= 1) {
+    const double c = ec[k + step - 1];
+    k = sx2 <= S * (c * fabs(c)) ? k + step : k;
   }
-  return lo;
+  return S == 0.0 ? 0 : k;
 }
 
 // The slot's bitstream (codes LSB first, code i at bits [i b, i b + b)) is

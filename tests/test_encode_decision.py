@@ -24,6 +24,11 @@ section 2.1).
    Restated here, and the record read back with the layout reader the GPU
    parity tests use (the chunk-major layout of the library header).
 
+3. The non-uniform encoder's search: per-angle edges from the library's host
+   tables, decided as x |x| <= S (c |c|) for either sign of c = cos theta by
+   steps 2^(b-1) .. 1; restated and compared with a scan of every edge under
+   the plain test and with the non-uniform oracle's codes off the cell edges.
+
 These are restatements of the kernel's steps (the kernel itself needs a GPU);
 what pins them is the oracle and the plain definitions, not the kernel.
 """
@@ -196,3 +201,63 @@ def test_slot_words_write_the_documented_layout(b):
     got, _, pads = helpers.unpack_records(rec[None, :], b)
     assert np.array_equal(got[0], codes)
     assert np.all(pads == 0)
+
+
+# ---------------------------------------------------------------- non-uniform
+
+def _polar_nu(x, S, ec, b):
+    """The non-uniform encoder's search (restated): the largest j with edge j
+    reached, x |x| <= S (c |c|) for c = cos theta_j, by steps 2^(b-1) .. 1."""
+    sx2 = x * abs(x)
+    k = 0
+    step = 1 << (b - 1)
+    while step >= 1:
+        c = ec[k + step - 1]
+        if sx2 <= S * (c * abs(c)):
+            k += step
+        step //= 2
+    return 0 if S == 0.0 else k
+
+
+def _polar_nu_scan(x, S, ec):
+    """Brute force with the plain test: phi >= theta <=> x <= sqrt(S) cos theta,
+    i.e. x <= 0 or x^2 <= S c^2 for c >= 0, x < 0 and x^2 >= S c^2 for c < 0."""
+    if S == 0.0:
+        return 0
+    best = 0
+    for j, c in enumerate(ec, start=1):
+        rhs = S * (c * c)
+        reach = (x <= 0.0 or x * x <= rhs) if c >= 0.0 else (x < 0.0 and x * x >= rhs)
+        if reach:
+            best = j
+    return best
+
+
+@pytest.mark.parametrize("b", [3, 4, 6, 8])
+def test_nonuniform_signed_square_search(b):
+    """The signed-square search equals the plain edge scan everywhere (ties and
+    zeros included) and the oracle's non-uniform codes off the cell edges."""
+    from compressed_kv_decode_ada_b200 import ops
+    from oracle import nonuniform as onu
+
+    ec, _, _ = ops.nonuniform_tables(D, b)
+    keys = _keys(12, seed=300 + b)
+    keys[0, 64:] = 0
+    keys[1, ::2] = keys[1, 1::2]
+    n = 1 << b
+    codes, _ = onu.encode(keys, b, 0.0, 0.05)
+    n_checked = 0
+    for t in range(keys.shape[0]):
+        x = oracle.bf16_to_f64(keys[t])
+        S = _suffix_sums(x)
+        phi = oracle.angles(x)
+        for i in range(126):
+            got = _polar_nu(x[i], S[i], ec[i], b)
+            assert got == _polar_nu_scan(x[i], S[i], ec[i]), (t, i)
+            pos = n * float(onu.polar_cdf(phi[i], D, i + 1))
+            if abs(pos - round(pos)) > 1e-9 * max(1.0, abs(pos)):
+                assert got == codes[t, i], (t, i, got, codes[t, i], pos)
+            n_checked += 1
+        # a zero input is the middle code: phi = pi / 2 sits on the middle edge
+        assert _polar_nu(0.0, 1.0, ec[0], b) == _polar_nu_scan(0.0, 1.0, ec[0])
+    assert n_checked == 12 * 126
