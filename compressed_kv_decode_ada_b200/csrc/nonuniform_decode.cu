@@ -197,23 +197,34 @@ __global__ void __launch_bounds__(kNuThreads) nu_decode_kernel(const NuParams p)
 #pragma unroll
       for (int c = 0; c < BITS; ++c) wv[c] = *reinterpret_cast<const uint4 *>(p.arena + rec + (c * 16 + slot) * 16);
       const float r = exp2f(fmaf((float)p.arena[rec + 256 * BITS + slot], Dh, Lh));
-      float f[G];
+      // two independent chains, angles 0 .. 63 (A) and 64 .. 126 (B, its
+      // products of sines started at 1), joined as f = A + P_A (B + u_q,127 P_B)
+      float fa[G], fb[G];
 #pragma unroll
-      for (int g = 0; g < G; ++g) f[g] = 0.0f;
-      float P = 1.0f;
-#pragma unroll
-      for (int j = 0; j < 127; ++j) {
+      for (int g = 0; g < G; ++g) fa[g] = fb[g] = 0.0f;
+      float Pa = 1.0f, Pb = 1.0f;
+      auto entry = [&](int j) -> float2 {
         const int e = j * N + (int)nu_code<BITS>(wv, j);
-        float2 cs;
-        if constexpr (kSmemTab) cs = stab[e];
-        else cs = __ldg(p.tab + e);
-        const float u = P * cs.x;
-        P *= cs.y;
+        if constexpr (kSmemTab) return stab[e];
+        else return __ldg(p.tab + e);
+      };
 #pragma unroll
-        for (int g = 0; g < G; ++g) f[g] = fmaf(uq[j][g], u, f[g]);
+      for (int j = 0; j < 64; ++j) {
+        const float2 ca = entry(j);
+        const float ua = Pa * ca.x;
+        Pa *= ca.y;
+#pragma unroll
+        for (int g = 0; g < G; ++g) fa[g] = fmaf(uq[j][g], ua, fa[g]);
+        if (j < 63) {
+          const float2 cb = entry(64 + j);
+          const float ub = Pb * cb.x;
+          Pb *= cb.y;
+#pragma unroll
+          for (int g = 0; g < G; ++g) fb[g] = fmaf(uq[64 + j][g], ub, fb[g]);
+        }
       }
 #pragma unroll
-      for (int g = 0; g < G; ++g) x[g] = qs[g] * r * fmaf(uq[127][g], P, f[g]);
+      for (int g = 0; g < G; ++g) x[g] = qs[g] * r * fmaf(Pa, fmaf(uq[127][g], Pb, fb[g]), fa[g]);
     }
     if (p.logits && t < t_end) {
 #pragma unroll
