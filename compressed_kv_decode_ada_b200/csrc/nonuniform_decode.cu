@@ -250,20 +250,30 @@ __global__ void __launch_bounds__(kNuThreads) nu_decode_kernel(const NuParams p)
       for (int k = 0; k < 4; ++k) acc[g][k] *= alpha;
       m[g] = mn;
     }
+    // P.V: lane l holds dims 4 l .. 4 l + 3; the chunk's value rows are
+    // loaded eight at a time before their products, so the loads overlap
     const unsigned okm = __ballot_sync(0xffffffffu, ok);
-    for (int i = 0; i < 32; ++i) {
-      if (!((okm >> i) & 1u)) continue;  // warp-uniform
-      const int pi = __shfl_sync(0xffffffffu, pid, i), si = __shfl_sync(0xffffffffu, slot, i);
-      const uint2 vr = *reinterpret_cast<const uint2 *>(p.v_pages + (((int64_t)pi * p.Hkv + h) * kPage + si) * kD +
-                                                         4 * lane);
-      const float v0 = bf16lo(vr.x), v1 = bf16hi(vr.x), v2 = bf16lo(vr.y), v3 = bf16hi(vr.y);
+    // this lane's token's value row (element offset), or -1
+    const int64_t vrow = ok ? (((int64_t)pid * p.Hkv + h) * kPage + slot) * kD : -1;
+    for (int i0 = 0; i0 < 32; i0 += 8) {
+      if (!((okm >> i0) & 0xffu)) continue;  // warp-uniform
+      uint2 vr[8];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float pg = __shfl_sync(0xffffffffu, pv[g], i);
-        acc[g][0] = fmaf(pg, v0, acc[g][0]);
-        acc[g][1] = fmaf(pg, v1, acc[g][1]);
-        acc[g][2] = fmaf(pg, v2, acc[g][2]);
-        acc[g][3] = fmaf(pg, v3, acc[g][3]);
+      for (int k = 0; k < 8; ++k) {
+        const int64_t o = __shfl_sync(0xffffffffu, vrow, i0 + k);
+        vr[k] = o >= 0 ? *reinterpret_cast<const uint2 *>(p.v_pages + o + 4 * lane) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float v0 = bf16lo(vr[k].x), v1 = bf16hi(vr[k].x), v2 = bf16lo(vr[k].y), v3 = bf16hi(vr[k].y);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float pg = __shfl_sync(0xffffffffu, pv[g], i0 + k);  // 0 for a token not decoded
+          acc[g][0] = fmaf(pg, v0, acc[g][0]);
+          acc[g][1] = fmaf(pg, v1, acc[g][1]);
+          acc[g][2] = fmaf(pg, v2, acc[g][2]);
+          acc[g][3] = fmaf(pg, v3, acc[g][3]);
+        }
       }
     }
   }
