@@ -145,3 +145,24 @@ def test_nonuniform_decode_matches_the_oracle(spkv, bits, kw):
             d = np.abs(got[sel] - ref[sel]) / np.maximum(scale, 1e-30)
             assert d.max() <= FB_TOL, d.max()
     assert err <= OUT_TOL, err
+
+
+@pytest.mark.parametrize("num_splits", [0, 3])
+def test_nonuniform_decode_long_context_splits(spkv, num_splits):
+    """A 5000-token context at b = 4 (G = 4): the default split count (about six
+    CTAs per SM: one page per split here) and three splits (each warp walks
+    many 32-token chunks, value rows batched eight at a time), against the
+    oracle and against each other."""
+    m = spkv[0]
+    wl, cache, (ec, mc, ms) = _build(spkv, 4, B=1, ctx=[5000], Hq=8, Hkv=2)
+    out = m.decode_attention_nonuniform(cache, wl.q, wl.block_table, wl.ctx_tensor(), wl.max_ctx, 4, ec, mc, ms,
+                                        num_splits=num_splits)
+    torch.cuda.synchronize()
+    assert cache.error_flags() == 0
+    out = out.cpu().numpy()
+    err = 0.0
+    for b, h in helpers.all_groups(wl):
+        oc, rc, L, D = _oracle_group(wl, b, h, 4)
+        want = onu.ada_group(wl.q_bits(b, h), oc, 4, rc, L, D, wl.values_bits(b, h), keep=wl.keep_of(b))
+        err = max(err, float(np.abs(out[b, h * wl.G:(h + 1) * wl.G] - want).max()))
+    assert err <= OUT_TOL, err
