@@ -12,11 +12,13 @@
 //   phi_i >= theta_k  <=>  x_i <= sqrt(S_i) cos(theta_k)
 // (S_i = sum_{j >= i} x_j^2) is decided from x_i^2 versus S_i cos^2(theta_k)
 // plus the signs.  The code is the largest k whose edge theta_k the angle
-// reaches (a binary search over the edges of the half of [0, pi] the sign of
-// x_i gives), i.e. floor(phi 2^b / pi) clamped to 2^b - 1 -- ties go to the
-// upper cell.  The azimuth (angle 127, range [0, 2 pi)) uses the same test on
-// (x_126, x_127) with the half-plane given by the sign of x_127.  The radius
-// code uses fp64 log2.  One thread encodes one key (spkv_encode.cuh).
+// reaches (a stepped search over the edges of the half of [0, pi] the sign of
+// x_i gives, one product and one comparison per step), i.e.
+// floor(phi 2^b / pi) clamped to 2^b - 1 -- ties go to the upper cell.  The
+// azimuth (angle 127, range [0, 2 pi)) uses the same test on (x_126, x_127)
+// with the half-plane given by the sign of x_127.  The radius code uses fp64
+// log2.  One thread encodes one key in bulk calls, one warp per key in small
+// ones (spkv_encode.cuh).
 #include "spkv_encode.cuh"
 
 namespace spkv {
@@ -117,9 +119,9 @@ __device__ __forceinline__ uint32_t enc_record(const EncodeParams &p, const EncP
 // The 32 key rows (8 KB, contiguous) come into the warp's shared-memory
 // stage with coalesced loads (rows 264 bytes apart, so the lanes' 8-byte
 // reads of their own rows fall in different bank pairs); each lane encodes
-// its key from there (encode_key_lane); the value rows are copied by the
-// whole warp, a row per instruction (coalesced 256-byte reads and writes),
-// eight rows in flight.
+// its key from there (encode_key_lane, reading two groups ahead); the value
+// rows are copied by the whole warp, a row per instruction (coalesced
+// 256-byte reads and writes), eight rows in flight.
 constexpr int kEncRowStride = 264;  // bytes per staged key row
 struct EncodeSmem {
   double pol_c2[kLutEntries];

@@ -1,7 +1,8 @@
 // spkv_encode.cuh -- a key into its page slot: one thread per key for the
-// bulk encode kernel (spkv_encode_keys), one warp per key for the decode
-// kernel's fused single-token append (spkv_decode_attention_append); the two
-// forms do the same arithmetic, so they write the same bytes for a key.
+// bulk encode kernel (spkv_encode_keys), one warp per key for small calls and
+// the decode kernel's fused single-token append (spkv_decode_attention_append);
+// the two forms make the same decisions with the same roundings, so they write
+// the same bytes for a key.
 //
 // Method: "SPHERICAL KV: Angle-Domain Attention and Rate-Distortion Retention
 // for Efficient Long-Context Inference", technical summary section 2.1
