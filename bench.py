@@ -577,8 +577,9 @@ def run_rdr(args):
 def run_profile_only(args):
     """One path alone, for profiler captures: W warm-up and K calls of
     'ada' (spkv_decode_attention), 'dense' (spkv_dense_decode), 'dtd'
-    (spkv_decompress_then_dot) or 'encode' (spkv_encode_keys of every context
-    key and value) on the workload, so a capture can skip and count its
+    (spkv_decompress_then_dot), 'encode' (spkv_encode_keys of every context
+    key and value), or the non-uniform quantiser's 'nu_decode' / 'nu_encode'
+    at b = 4 on the workload, so a capture can skip and count its
     launches exactly.  Prints one JSON line with the mean CUDA-event time."""
     import torch
 
@@ -608,6 +609,25 @@ def run_profile_only(args):
         fn = lambda: spkv.decompress_then_dot(cache, ks, wl.q, wl.block_table, ctx, max_ctx, ws=ws,
                                               num_splits=args.splits, stream=stream)
         per_call = ["decompress_kernel", "split_kernel (dense)", "merge_kernel"]
+    elif path in ("nu_decode", "nu_encode"):
+        # the non-uniform quantiser at b = 4: its own cache of the workload
+        ec, mc, msn = (torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in spkv.nonuniform_tables(128, 4))
+        cache = spkv.SpkvCache(wl.num_pages, wl.Hkv, np.full(wl.num_pages, 4, np.int64), wl.rad_lo, wl.rad_step,
+                               device=dev, keep_mask=wl.keep_mask)
+        n0 = int(wl.ctx[0])
+        if len(set(int(c) for c in wl.ctx)) != 1:
+            raise SystemExit("--profile-only nu_*: a workload with equal context lengths")
+        kv, vv = wl.keys.view(wl.B, n0, wl.Hkv, -1), wl.values.view(wl.B, n0, wl.Hkv, -1)
+        zero = torch.zeros(wl.B, dtype=torch.int32, device=dev)
+        enc = lambda: spkv.encode_keys_nonuniform(cache, kv, zero, wl.block_table, 4, ec, values=vv, stream=stream)
+        enc()
+        if path == "nu_encode":
+            fn = enc
+            per_call = ["encode_kernel (non-uniform)"]
+        else:
+            fn = lambda: spkv.decode_attention_nonuniform(cache, wl.q, wl.block_table, ctx, max_ctx, 4, ec, mc, msn,
+                                                          stream=stream)
+            per_call = ["nu_table_kernel", "nu_decode_kernel", "merge_partials_kernel"]
     else:
         fn = lambda: workload.prefill(cache, wl)
         per_call = ["encode_kernel"]
@@ -643,7 +663,8 @@ def main():
                     help="also time the other full-size workloads (128K, 70B shape, ragged mixed tiers)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-only", choices=["ada", "dense", "dtd", "encode"], default=None,
+    ap.add_argument("--profile-only", choices=["ada", "dense", "dtd", "encode", "nu_decode", "nu_encode"],
+                    default=None,
                     help="run one path alone, --warmup + --steps calls (one JSON line; profiler captures)")
     ap.add_argument("--rdr", action="store_true",
                     help="time only spkv_rdr_plan on the workload's keys (one JSON line; profiler captures)")
