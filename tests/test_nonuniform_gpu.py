@@ -192,3 +192,46 @@ def test_nonuniform_full_size_sampled_parity(spkv):
     assert err <= OUT_TOL, err
     vmax = wl.values.float().abs().amax().item()
     assert outn.max() <= vmax + 1e-3 and outn.min() >= -vmax - 1e-3
+
+
+def test_nonuniform_edge_cases(spkv):
+    """Empty and fully evicted sequences give 0, a bad page id and a page of
+    another width set their device-error bits without a fault, and the
+    untouched sequences keep their parity."""
+    m = spkv[0]
+    wl, cache, (ec, mc, ms) = _build(spkv, 4, B=3, ctx=[0, 40, 300], Hq=4, Hkv=1)
+    km = cache.keep_mask if cache.keep_mask is not None else torch.full(
+        (wl.num_pages, wl.Hkv), -1, dtype=torch.int16, device="cuda")
+    km[torch.as_tensor(wl.block_table_np[1, :3], device="cuda").long()] = 0  # evict sequence 1
+    cache.keep_mask = km
+
+    def dec(bt):
+        out = m.decode_attention_nonuniform(cache, wl.q, bt, wl.ctx_tensor(), wl.max_ctx, 4, ec, mc, ms)
+        torch.cuda.synchronize()
+        return out
+
+    out = dec(wl.block_table).cpu().numpy()
+    assert cache.error_flags() == 0
+    assert np.all(out[0] == 0) and np.all(out[1] == 0)
+    oc, rc, L, D = _oracle_group(wl, 2, 0, 4)
+    want = onu.ada_group(wl.q_bits(2, 0), oc, 4, rc, L, D, wl.values_bits(2, 0), keep=wl.keep_of(2))
+    assert np.abs(out[2] - want).max() <= OUT_TOL
+    # a page id past the pool: flagged, skipped, no fault
+    bt = wl.block_table.clone()
+    bt[2, 3] = wl.num_pages + 7
+    cache.clear_errors()
+    out = dec(bt)
+    assert cache.error_flags() & 1
+    assert torch.isfinite(out).all()
+    # a page written at another width: flagged
+    hdr = cache.hdr.clone()
+    cache.hdr[int(wl.block_table_np[2, 0]), 4] = 6
+    cache.clear_errors()
+    out = dec(wl.block_table)
+    assert cache.error_flags() & 2
+    assert torch.isfinite(out).all()
+    cache.hdr.copy_(hdr)
+    # B = 0 is a no-op
+    m.decode_attention_nonuniform(cache, wl.q[:0], wl.block_table[:0], wl.ctx_tensor()[:0], wl.max_ctx, 4, ec, mc,
+                                  ms)
+    torch.cuda.synchronize()
